@@ -1,0 +1,162 @@
+"""ctypes front end of the fp64 CPU oracle (``oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU-baseline leg use it; the
+product path never does.  Inputs are the raw bf16 bit patterns (numpy uint16) that the CUDA path
+receives; outputs are float64 numpy arrays.
+
+Every function here applies the plain attention definition (see the header of ``oracle.c`` for the
+passages it follows); the pins that tie it to what the pages and the mathematics fix live in
+``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_dbl = ctypes.c_double
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` with gcc into ``liboracle.so`` beside it (plain -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math",
+                               "-o", _LIB, _SRC, "-lm", "-lpthread"])
+    return _LIB
+
+
+class OracleLib:
+    """The oracle's entry points bound to one compiled library (the default one, or a test build)."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        lib.oracle_attention.argtypes = [_u16p, _u16p, _u16p, _i64, _i64, _int, _int, _dbl,
+                                         _f64p, _f64p, _int]
+        lib.oracle_attention_rows.argtypes = [_u16p, _u16p, _u16p, _i64, _int, _int, _dbl, _i64p,
+                                              _i64, _f64p, _f64p, _int]
+        lib.oracle_attention_probs.argtypes = [_u16p, _u16p, _i64, _int, _int, _dbl, _f64p]
+        lib.oracle_flash_alg1.argtypes = [_u16p, _u16p, _u16p, _i64, _int, _int, _dbl, _int, _int,
+                                          _f64p, _f64p, _f64p]
+        lib.oracle_decode_paged.argtypes = [_u16p, _u16p, _u16p, _i32p, _int, _i32p, _int, _int,
+                                            _int, _int, _dbl, _f64p, _f64p, _int]
+        for f in (lib.oracle_attention, lib.oracle_attention_rows, lib.oracle_attention_probs,
+                  lib.oracle_flash_alg1, lib.oracle_decode_paged):
+            f.restype = ctypes.c_int
+        self.lib = lib
+        self.path = path
+
+    def attention(self, q, k, v, causal: bool, scale: float, nthreads: int | None = None):
+        """All rows. q, k, v: uint16 [..., N, d] (bf16 bits). Returns (o [..., N, d], lse [..., N])."""
+        q, k, v = _bits(q), _bits(k), _bits(v)
+        *lead, N, d = q.shape
+        BH = int(np.prod(lead)) if lead else 1
+        o = np.empty((BH, N, d), np.float64)
+        lse = np.empty((BH, N), np.float64)
+        rc = self.lib.oracle_attention(q, k, v, BH, N, d, int(causal), scale, o, lse,
+                                       nthreads or default_threads())
+        if rc:
+            raise ValueError("oracle_attention: bad arguments")
+        return o.reshape(*lead, N, d), lse.reshape(*lead, N)
+
+    def attention_rows(self, q, k, v, causal: bool, scale: float, pairs, nthreads: int | None = None):
+        """Selected rows. q, k, v: uint16 [..., N, d] (leading dims flattened to bh); pairs: int64
+        [n, 2] of (bh, row).  Returns (o [n, d], lse [n])."""
+        q, k, v = _bits(q), _bits(k), _bits(v)
+        N, d = q.shape[-2], q.shape[-1]
+        pairs = np.ascontiguousarray(pairs, dtype=np.int64).reshape(-1, 2)
+        n = pairs.shape[0]
+        o = np.empty((n, d), np.float64)
+        lse = np.empty((n,), np.float64)
+        rc = self.lib.oracle_attention_rows(q, k, v, N, d, int(causal), scale, pairs, n, o, lse,
+                                            nthreads or default_threads())
+        if rc:
+            raise ValueError("oracle_attention_rows: bad arguments")
+        return o, lse
+
+    def probs(self, q, k, causal: bool, scale: float):
+        """Full probability matrix P [N, N] of one head (masked entries 0)."""
+        q, k = _bits(q), _bits(k)
+        N, d = q.shape
+        P = np.empty((N, N), np.float64)
+        self.lib.oracle_attention_probs(q, k, N, d, int(causal), scale, P)
+        return P
+
+    def flash_alg1(self, q, k, v, causal: bool, scale: float, Br: int, Bc: int):
+        """The tiled algorithm with block sizes Br x Bc on one head. Returns (O, l, m)."""
+        q, k, v = _bits(q), _bits(k), _bits(v)
+        N, d = q.shape
+        O = np.empty((N, d), np.float64)
+        l = np.empty((N,), np.float64)
+        m = np.empty((N,), np.float64)
+        rc = self.lib.oracle_flash_alg1(q, k, v, N, d, int(causal), scale, Br, Bc, O, l, m)
+        if rc:
+            raise ValueError("oracle_flash_alg1: bad arguments")
+        return O, l, m
+
+    def decode_paged(self, q, k_pool, v_pool, block_table, seq_lens, scale: float, page: int = 16,
+                     nthreads: int | None = None):
+        """q [S,H,d]; pools [P,H,page,d] (uint16 bf16 bits); block_table int32 [S,max_blocks];
+        seq_lens int32 [S].  Returns (o [S,H,d], lse [S,H])."""
+        q, k_pool, v_pool = _bits(q), _bits(k_pool), _bits(v_pool)
+        table = np.ascontiguousarray(block_table, dtype=np.int32)
+        lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        S, H, d = q.shape
+        o = np.empty((S, H, d), np.float64)
+        lse = np.empty((S, H), np.float64)
+        rc = self.lib.oracle_decode_paged(q, k_pool, v_pool, table, table.shape[1], lens, S, H, d,
+                                          page, scale, o, lse, nthreads or default_threads())
+        if rc:
+            raise ValueError("oracle_decode_paged: bad arguments")
+        return o, lse
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _bits(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns (uint16)")
+    return a
+
+
+def default() -> OracleLib:
+    """The oracle built from ``oracle.c`` as committed."""
+    global _lib
+    if _lib is None:
+        _lib = OracleLib(build())
+    return _lib
+
+
+def attention(*a, **kw):
+    return default().attention(*a, **kw)
+
+
+def attention_rows(*a, **kw):
+    return default().attention_rows(*a, **kw)
+
+
+def probs(*a, **kw):
+    return default().probs(*a, **kw)
+
+
+def flash_alg1(*a, **kw):
+    return default().flash_alg1(*a, **kw)
+
+
+def decode_paged(*a, **kw):
+    return default().decode_paged(*a, **kw)

@@ -1,0 +1,267 @@
+"""Pins that tie the fp64 oracle to what the pages and the mathematics fix, independently of the
+oracle's own code.  Each pin takes an ``OracleLib`` and raises AssertionError when it does not hold,
+so the same checks run against the committed oracle (test_oracle_pins.py) and against builds of it
+with a planted mistake (test_oracle_mutants.py), which must each fail at least one pin.
+
+The facts used:
+* softmax rows are weights that sum to one ("FlashAttention-2 GPU work partitioning", section 2);
+* attention is softmax(Q K^T * scale) V with scale = 1 / sqrt(d_k) ("LLM study notes",
+  self-attention steps), so: equal scores give the mean of V; one key gives that key's value;
+  a dominant score selects its value row; two keys reduce to the logistic function; a constant
+  added to a score row changes nothing but the log-sum-exp; the result is equivariant under
+  permutations and linear in V;
+* the causal mask shows query i only keys 0..i ("FlashAttention-2 GPU work partitioning", section 4);
+* the tiled algorithm of "Flash Attention" (myungum), section 2, computes exact attention, so any
+  block sizes give the plain result;
+* a paged KV cache is only a relocation of logically contiguous rows ("LLM study notes", paged
+  attention).
+Reference values are formed with numpy/scipy from the widened inputs, never from the oracle.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import scipy.special as sps
+import torch
+
+import workloads as W
+
+
+def bf16(x) -> np.ndarray:
+    """Round to bf16 and return the raw bits (uint16)."""
+    t = torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def widen(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def rnd(shape, seed, tid=W.TID_Q) -> np.ndarray:
+    n = int(np.prod(shape))
+    return W.bf16_bits(W.normal_bf16(seed, tid, n)).reshape(shape)
+
+
+def close(a, b, tol, what):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert np.all(np.isfinite(a)) and err <= tol, f"{what}: max err {err} > {tol}"
+
+
+# ------------------------------------------------------------------------------------------------
+
+def pin_uniform_scores(orc):
+    """Q = 0: every visible key gets the same weight, so O_i = mean of the visible V rows and
+    LSE_i = ln |A_i| (ln N, or ln(i+1) when causal)."""
+    N, d = 37, 16
+    q = bf16(np.zeros((N, d)))
+    k = rnd((N, d), 1, W.TID_K)
+    v = rnd((N, d), 1, W.TID_V)
+    V = widen(v)
+    for causal in (False, True):
+        o, lse = orc.attention(q, k, v, causal, 0.25)
+        for i in range(N):
+            n = i + 1 if causal else N
+            close(o[i], V[:n].mean(axis=0), 1e-13, f"uniform O row {i} causal={causal}")
+            close(lse[i], math.log(n), 1e-13, f"uniform LSE row {i} causal={causal}")
+
+
+def pin_single_key(orc):
+    """N = 1: O = V and LSE = scale * q.k; and causal row 0 (only key 0 visible) for any N."""
+    d = 24
+    q = rnd((1, d), 2)
+    k = rnd((1, d), 2, W.TID_K)
+    v = rnd((1, d), 2, W.TID_V)
+    scale = 0.3
+    for causal in (False, True):
+        o, lse = orc.attention(q, k, v, causal, scale)
+        close(o[0], widen(v)[0], 1e-15, "N=1 O")
+        close(lse[0], scale * float(widen(q)[0] @ widen(k)[0]), 1e-12, "N=1 LSE")
+    N = 19
+    q = rnd((N, d), 3)
+    k = rnd((N, d), 3, W.TID_K)
+    v = rnd((N, d), 3, W.TID_V)
+    o, lse = orc.attention(q, k, v, True, scale)
+    close(o[0], widen(v)[0], 1e-15, "causal row 0 O")
+    close(lse[0], scale * float(widen(q)[0] @ widen(k)[0]), 1e-12, "causal row 0 LSE")
+
+
+def pin_dominant_score(orc):
+    """Orthogonal keys c e_j and queries c e_t: the score gap scale*c^2 (> 60) makes the softmax
+    one-hot, so O_t = V_t within exp(-60) and LSE_t = scale c^2 (+ a term below 1e-25)."""
+    N = d = 8
+    c = 32.0
+    scale = 1.0 / math.sqrt(d)
+    k = bf16(c * np.eye(N, d))
+    v = rnd((N, d), 4, W.TID_V)
+    perm = np.array([3, 0, 7, 5, 1, 6, 2, 4])
+    q = bf16(c * np.eye(N, d)[perm])
+    o, lse = orc.attention(q, k, v, False, scale)
+    for i in range(N):
+        close(o[i], widen(v)[perm[i]], 1e-20 + 1e-12, f"one-hot O row {i}")
+        close(lse[i], scale * c * c, 1e-12, f"one-hot LSE row {i}")
+
+
+def pin_two_keys_logistic(orc):
+    """N = 2 reduces to the logistic function: row i gets weight sigma(s_i0 - s_i1) on v_0 and
+    sigma(s_i1 - s_i0) on v_1; LSE = max + log1p(exp(-|s_0 - s_1|)).  The causal row 0 sees v_0."""
+    d = 32
+    q = rnd((2, d), 5)
+    k = rnd((2, d), 5, W.TID_K)
+    v = rnd((2, d), 5, W.TID_V)
+    scale = 0.2
+    Q, K, V = widen(q), widen(k), widen(v)
+    s = scale * (Q @ K.T)
+    sig = lambda x: 1.0 / (1.0 + math.exp(-x))
+    o, lse = orc.attention(q, k, v, False, scale)
+    for i in range(2):
+        a = sig(s[i, 0] - s[i, 1])
+        close(o[i], a * V[0] + (1 - a) * V[1], 1e-13, f"logistic O row {i}")
+        close(lse[i], max(s[i]) + math.log1p(math.exp(-abs(s[i, 0] - s[i, 1]))), 1e-13,
+              f"logistic LSE row {i}")
+    o, lse = orc.attention(q, k, v, True, scale)
+    a = sig(s[1, 0] - s[1, 1])
+    close(o[1], a * V[0] + (1 - a) * V[1], 1e-13, "logistic causal O row 1")
+    close(o[0], V[0], 1e-15, "logistic causal O row 0")
+
+
+def pin_shift_invariance(orc):
+    """K' = K + 1 u^T adds scale*(q_i . u) to every score of row i: O is unchanged and LSE moves by
+    that amount.  Small integers keep K' exact in bf16."""
+    rng = np.random.default_rng(6)
+    N, d = 23, 8
+    Q = rng.integers(-3, 4, (N, d)).astype(np.float64)
+    K = rng.integers(-3, 4, (N, d)).astype(np.float64)
+    V = rng.integers(-5, 6, (N, d)).astype(np.float64)
+    u = rng.integers(-2, 3, (d,)).astype(np.float64)
+    scale = 0.125
+    for causal in (False, True):
+        o1, l1 = orc.attention(bf16(Q), bf16(K), bf16(V), causal, scale)
+        o2, l2 = orc.attention(bf16(Q), bf16(K + u[None, :]), bf16(V), causal, scale)
+        close(o2, o1, 1e-12, f"shift O causal={causal}")
+        close(l2, l1 + scale * (Q @ u), 1e-12, f"shift LSE causal={causal}")
+
+
+def pin_rows_sum_to_one(orc):
+    """Every row of P sums to 1 and masked entries are 0; P matches scipy's softmax of Q K^T*scale."""
+    N, d = 64, 16
+    q = rnd((N, d), 7)
+    k = rnd((N, d), 7, W.TID_K)
+    scale = 0.25
+    S = scale * (widen(q) @ widen(k).T)
+    for causal in (False, True):
+        P = orc.probs(q, k, causal, scale)
+        close(P.sum(axis=1), np.ones(N), 1e-14, f"row sums causal={causal}")
+        if causal:
+            assert np.all(P[np.triu_indices(N, 1)] == 0.0), "masked entries of P are not zero"
+            S = S.copy()
+            S[np.triu_indices(N, 1)] = -np.inf
+        close(P, sps.softmax(S, axis=1), 1e-14, f"P vs scipy softmax causal={causal}")
+
+
+def pin_library_softmax(orc):
+    """O = softmax(S) V and LSE = logsumexp(S) formed with numpy/scipy on the widened inputs."""
+    B_H, N, d = 3, 41, 16
+    q = rnd((B_H, N, d), 8)
+    k = rnd((B_H, N, d), 8, W.TID_K)
+    v = rnd((B_H, N, d), 8, W.TID_V)
+    scale = 1 / 4
+    Q, K, V = widen(q), widen(k), widen(v)
+    for causal in (False, True):
+        o, lse = orc.attention(q, k, v, causal, scale)
+        for bh in range(B_H):
+            S = scale * Q[bh] @ K[bh].T
+            if causal:
+                S[np.triu_indices(N, 1)] = -np.inf
+            close(o[bh], sps.softmax(S, axis=1) @ V[bh], 1e-13, f"scipy O causal={causal}")
+            close(lse[bh], sps.logsumexp(S, axis=1), 1e-13, f"scipy LSE causal={causal}")
+
+
+def pin_permutation(orc):
+    """Non-causal: permuting K and V rows together leaves O unchanged; permuting Q rows permutes O."""
+    N, d = 29, 8
+    q = rnd((N, d), 9)
+    k = rnd((N, d), 9, W.TID_K)
+    v = rnd((N, d), 9, W.TID_V)
+    p = np.random.default_rng(9).permutation(N)
+    o, lse = orc.attention(q, k, v, False, 0.35)
+    o2, lse2 = orc.attention(q, k[p].copy(), v[p].copy(), False, 0.35)
+    close(o2, o, 1e-13, "permute K,V")
+    close(lse2, lse, 1e-13, "permute K,V LSE")
+    o3, lse3 = orc.attention(q[p].copy(), k, v, False, 0.35)
+    close(o3, o[p], 1e-15, "permute Q")
+    close(lse3, lse[p], 1e-15, "permute Q LSE")
+
+
+def pin_linear_in_v(orc):
+    """O(Q, K, aV + bV') = a O(Q, K, V) + b O(Q, K, V'); integer V, V' keep aV + bV' exact."""
+    rng = np.random.default_rng(10)
+    N, d = 31, 8
+    q = rnd((N, d), 10)
+    k = rnd((N, d), 10, W.TID_K)
+    V1 = rng.integers(-4, 5, (N, d)).astype(np.float64)
+    V2 = rng.integers(-4, 5, (N, d)).astype(np.float64)
+    for causal in (False, True):
+        o1, _ = orc.attention(q, k, bf16(V1), causal, 0.3)
+        o2, _ = orc.attention(q, k, bf16(V2), causal, 0.3)
+        o3, _ = orc.attention(q, k, bf16(2 * V1 - 3 * V2), causal, 0.3)
+        close(o3, 2 * o1 - 3 * o2, 1e-12, f"linear in V causal={causal}")
+
+
+def pin_tiled_algorithm(orc):
+    """The tiled algorithm (outer loop over K/V blocks, running m and l, O renormalised each step)
+    equals the plain definition for any block sizes, ragged tails included; LSE = m + ln l."""
+    N, d = 45, 16
+    q = rnd((N, d), 11)
+    k = rnd((N, d), 11, W.TID_K)
+    v = rnd((N, d), 11, W.TID_V)
+    scale = 0.25
+    for causal in (False, True):
+        o, lse = orc.attention(q, k, v, causal, scale)
+        for Br, Bc in ((1, 1), (3, 5), (7, 3), (16, 16), (45, 45), (64, 8), (5, 64)):
+            O, l, m = orc.flash_alg1(q, k, v, causal, scale, Br, Bc)
+            close(O, o, 1e-12, f"tiled O Br={Br} Bc={Bc} causal={causal}")
+            close(m + np.log(l), lse, 1e-12, f"tiled LSE Br={Br} Bc={Bc} causal={causal}")
+
+
+def pin_paged_decode(orc):
+    """Paged decode = plain attention over the sequence's rows gathered in logical order = the last
+    row of causal attention over those rows; shuffling the pool with the table changes nothing."""
+    case = W.DecodeCase("pin", S=3, H=2, d=16, lens=[1, 17, 40])
+    inp = W.make_decode(case)
+    q = W.bf16_bits(inp["q"])
+    kp = W.bf16_bits(inp["k_pool"])
+    vp = W.bf16_bits(inp["v_pool"])
+    table = inp["block_table"].numpy()
+    lens = inp["seq_lens"].numpy()
+    o, lse = orc.decode_paged(q, kp, vp, table, lens, case.scale)
+    for s, L in enumerate(case.lens):
+        for h in range(case.H):
+            rows = [(int(table[s, t // 16]), t % 16) for t in range(L)]
+            Kc = np.stack([kp[b, h, r] for b, r in rows])
+            Vc = np.stack([vp[b, h, r] for b, r in rows])
+            Qc = np.concatenate([np.zeros((L - 1, case.d), np.uint16), q[s, h][None]], axis=0)
+            oc, lc = orc.attention(Qc, Kc, Vc, True, case.scale)
+            close(o[s, h], oc[-1], 1e-13, f"paged vs causal last row s={s} h={h}")
+            close(lse[s, h], lc[-1], 1e-13, f"paged vs causal last row LSE s={s} h={h}")
+            S = case.scale * widen(Kc) @ widen(q[s, h])
+            close(o[s, h], sps.softmax(S) @ widen(Vc), 1e-13, f"paged vs scipy s={s} h={h}")
+    # relocate: move every physical block b to position pi(b), rewrite the table
+    P = kp.shape[0]
+    pi = np.random.default_rng(12).permutation(P)
+    kp2 = np.empty_like(kp)
+    vp2 = np.empty_like(vp)
+    kp2[pi] = kp
+    vp2[pi] = vp
+    t2 = np.where(table >= 0, pi[np.maximum(table, 0)], -1).astype(np.int32)
+    o2, lse2 = orc.decode_paged(q, kp2, vp2, t2, lens, case.scale)
+    close(o2, o, 0.0, "relocated pool O")
+    close(lse2, lse, 0.0, "relocated pool LSE")
+
+
+ALL_PINS = [pin_uniform_scores, pin_single_key, pin_dominant_score, pin_two_keys_logistic,
+            pin_shift_invariance, pin_rows_sum_to_one, pin_library_softmax, pin_permutation,
+            pin_linear_in_v, pin_tiled_algorithm, pin_paged_decode]
