@@ -1,0 +1,183 @@
+"""Exact attention forward for NVIDIA B200 (sm_100a): Python binding of ``libfa_b200.so``.
+
+The functions here only marshal arguments (pointers, sizes, the current CUDA stream) into the C ABI
+of include/fa.h; every step of the attention runs in the library's CUDA kernels.  PyTorch supplies
+device memory and streams.  There is no fallback: if the library is missing or the device is not
+an sm_100 GPU, calls raise.
+
+    o, lse = fa_fwd(q, k, v, causal=True)            # q, k, v: bf16 [B, H, N, d] on cuda
+    o, lse = fa_decode_paged(q, k_pool, v_pool, block_table, seq_lens)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+__all__ = ["fa_fwd", "fa_decode_paged", "fa_decode_workspace_size", "device_status",
+           "FaError", "library_path", "load_library", "EXPORTED_SYMBOLS", "STATUS"]
+
+STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_ALIGNMENT",
+          4: "FA_ERR_LAUNCH", 5: "FA_ERR_TIMEOUT", 6: "FA_ERR_WORKSPACE"}
+FA_OUT_BF16, FA_OUT_F32 = 0, 1
+
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
+                    "fa_get_device_status", "fa_status_string", "fa_last_error_string",
+                    "fa_version")
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {STATUS.get(status, status)}"
+        if _lib is not None:
+            msg = f"{where}: {_lib.fa_status_string(status).decode()}"
+            if status == 4:
+                msg += f" ({_lib.fa_last_error_string().decode()})"
+        super().__init__(msg)
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load_library():
+    """Load the in-tree shared library (build it first with ``python -m exact_attention_158_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(f"CUDA library not built: {path} is missing "
+                          "(run `python -m exact_attention_158_b200.build`)")
+    lib = ctypes.CDLL(path)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, f32, vp]
+    lib.fa_fwd.restype = i32
+    lib.fa_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.fa_decode_workspace_size.restype = sz
+    lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, i32, vp, i32, i32, i32, f32,
+                                    vp, sz, vp]
+    lib.fa_decode_paged.restype = i32
+    lib.fa_get_device_status.argtypes = [vp]
+    lib.fa_get_device_status.restype = i32
+    lib.fa_status_string.argtypes = [i32]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_last_error_string.argtypes = []
+    lib.fa_last_error_string.restype = ctypes.c_char_p
+    lib.fa_version.argtypes = []
+    lib.fa_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise FaError(status, where)
+
+
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _require(t: torch.Tensor, name: str, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _out_code(out_dtype) -> int:
+    if out_dtype == torch.bfloat16:
+        return FA_OUT_BF16
+    if out_dtype == torch.float32:
+        return FA_OUT_F32
+    raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+
+
+def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None,
+           out_dtype=torch.bfloat16, out=None, lse=None, return_lse: bool = True, stream=None):
+    """Exact attention forward.  q, k, v: bf16 [B, H, N, d] contiguous on one CUDA device.
+
+    Returns (o [B, H, N, d] in out_dtype, lse fp32 [B, H, N] or None)."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one shape [B, H, N, d]")
+    B, H, N, d = q.shape
+    code = _out_code(out_dtype)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    else:
+        _require(out, "out", out_dtype)
+        if out.shape != q.shape:
+            raise ValueError("out has the wrong shape")
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _require(lse, "lse", torch.float32)
+        if lse.shape != (B, H, N):
+            raise ValueError("lse has the wrong shape")
+    with torch.cuda.device(q.device):
+        st = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), code,
+                        lse.data_ptr() if lse is not None else None, B, H, N, d, int(causal),
+                        float(scale) if scale is not None else 0.0, _stream_handle(stream))
+    _check(st, "fa_fwd")
+    return out, lse
+
+
+def fa_decode_workspace_size(num_seqs: int, H: int, d: int, max_blocks_per_seq: int) -> int:
+    return int(load_library().fa_decode_workspace_size(num_seqs, H, d, max_blocks_per_seq))
+
+
+def fa_decode_paged(q, k_pool, v_pool, block_table, seq_lens, scale: float | None = None,
+                    out_dtype=torch.bfloat16, out=None, lse=None, return_lse: bool = True,
+                    workspace=None, stream=None):
+    """One decode step over a paged KV cache.
+
+    q bf16 [S, H, d]; k_pool, v_pool bf16 [num_blocks, H, 16, d]; block_table int32
+    [S, max_blocks]; seq_lens int32 [S].  Returns (o [S, H, d], lse fp32 [S, H] or None)."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _require(t, n)
+    _require(block_table, "block_table", torch.int32)
+    _require(seq_lens, "seq_lens", torch.int32)
+    S, H, d = q.shape
+    P = k_pool.shape[0]
+    if k_pool.shape != (P, H, 16, d) or v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool / v_pool must be [num_blocks, H, 16, d]")
+    if block_table.dim() != 2 or block_table.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_table must be [S, max_blocks] and seq_lens [S]")
+    maxb = block_table.shape[1]
+    code = _out_code(out_dtype)
+    if out is None:
+        out = torch.empty((S, H, d), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((S, H), dtype=torch.float32, device=q.device)
+    need = lib.fa_decode_workspace_size(S, H, d, maxb)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib.fa_decode_paged(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                 block_table.data_ptr(), maxb, seq_lens.data_ptr(), P,
+                                 out.data_ptr(), code,
+                                 lse.data_ptr() if lse is not None else None, S, H, d,
+                                 float(scale) if scale is not None else 0.0,
+                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                 _stream_handle(stream))
+    _check(st, "fa_decode_paged")
+    return out, lse
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the library's device status word."""
+    return int(load_library().fa_get_device_status(_stream_handle(stream)))

@@ -1,0 +1,283 @@
+// fa_lib.cu -- the C ABI declared in include/fa.h: argument checks, TMA descriptors, launches.
+// Host code only decides shapes and launches; every step of the attention itself runs in the
+// kernels of fa_prefill.cuh and fa_decode.cuh.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "fa.h"
+#include "fa_decode.cuh"
+#include "fa_prefill.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+
+thread_local std::string t_last_error;
+
+fa_status launch_failed(cudaError_t e) {
+  t_last_error = cudaGetErrorString(e);
+  return FA_ERR_LAUNCH;
+}
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int num_sms = 0;
+  bool prefill_attr[2] = {false, false};
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+
+// Looks up (once per device) whether the current device is an sm_100 part and its SM count.
+fa_status current_device(DeviceInfo **out, int *dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return launch_failed(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo &d = g_devices[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return launch_failed(e);
+    d.supported = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    d.probed = true;
+  }
+  if (!d.supported) return FA_ERR_UNSUPPORTED;
+  *out = &d;
+  *dev_out = dev;
+  return FA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [BH, N, d] bf16 viewed as a 3-D tensor (d innermost); boxes of 64 x 128 x 1 with 128-byte
+// swizzle, rows past N read as zeros.
+bool encode_bhnd(CUtensorMap *map, const void *base, int d, int N, int BH) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+bool resolve_scale(float scale, int d, float *out) {
+  if (std::isnan(scale) || std::isinf(scale)) return false;
+  *out = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+  return true;
+}
+
+template <int HD>
+fa_status launch_prefill(DeviceInfo &dev, const void *q, const void *k, const void *v, void *o,
+                         int o_f32, float *lse, int BH, int N, int causal, float scale,
+                         cudaStream_t stream) {
+  using C = fa::PrefillCfg<HD>;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bhnd(&tq, q, HD, N, BH) || !encode_bhnd(&tk, k, HD, N, BH) ||
+      !encode_bhnd(&tv, v, HD, N, BH)) {
+    t_last_error = "cuTensorMapEncodeTiled failed";
+    return FA_ERR_LAUNCH;
+  }
+  fa::PrefillParams p;
+  p.o = o;
+  p.lse = lse;
+  p.o_f32 = o_f32;
+  p.BH = BH;
+  p.N = N;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_pairs = (N + 2 * fa::kBM - 1) / (2 * fa::kBM);
+  p.num_super = causal ? BH * ((p.num_pairs + 1) / 2) : BH * p.num_pairs;
+  const int slot = HD == 128 ? 1 : 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!dev.prefill_attr[slot]) {
+      cudaError_t e = cudaFuncSetAttribute(fa::fa_prefill_kernel<HD>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(C::kSmemBytes));
+      if (e != cudaSuccess) return launch_failed(e);
+      dev.prefill_attr[slot] = true;
+    }
+  }
+  const int grid = p.num_super < dev.num_sms ? p.num_super : dev.num_sms;
+  fa::fa_prefill_kernel<HD><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : launch_failed(e);
+}
+
+int decode_splits(int max_blocks) {
+  return (max_blocks + fa::kDecodeChunkPages - 1) / fa::kDecodeChunkPages;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, fa_out_dtype o_dtype,
+                 float *lse, int B, int H, int N, int d, int causal, float scale,
+                 fa_stream_t stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  float sc;
+  if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  const int BH = B * H;
+  const size_t rows = static_cast<size_t>(BH) * N;
+  const size_t in_bytes = rows * d * 2;
+  const size_t o_bytes = rows * d * (o_dtype == FA_OUT_F32 ? 4 : 2);
+  if (overlaps(o, o_bytes, q, in_bytes) || overlaps(o, o_bytes, k, in_bytes) ||
+      overlaps(o, o_bytes, v, in_bytes))
+    return FA_ERR_INVALID_ARG;
+  if (lse && (overlaps(lse, rows * 4, q, in_bytes) || overlaps(lse, rows * 4, k, in_bytes) ||
+              overlaps(lse, rows * 4, v, in_bytes) || overlaps(lse, rows * 4, o, o_bytes)))
+    return FA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  const int o_f32 = o_dtype == FA_OUT_F32;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128) return launch_prefill<128>(*dev, q, k, v, o, o_f32, lse, BH, N, causal, sc, s);
+  return launch_prefill<64>(*dev, q, k, v, o, o_f32, lse, BH, N, causal, sc, s);
+}
+
+size_t fa_decode_workspace_size(int num_seqs, int H, int d, int max_blocks_per_seq) {
+  if (num_seqs < 1 || H < 1 || max_blocks_per_seq < 1 || (d != 64 && d != 128)) return 0;
+  const size_t units = static_cast<size_t>(num_seqs) * H * decode_splits(max_blocks_per_seq);
+  return units * (d + 2) * sizeof(float);
+}
+
+fa_status fa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
+                          const int32_t *block_table, int max_blocks_per_seq,
+                          const int32_t *seq_lens, int num_blocks, void *o, fa_out_dtype o_dtype,
+                          float *lse, int S, int H, int d, float scale, void *workspace,
+                          size_t workspace_bytes, fa_stream_t stream) {
+  if (!q || !k_pool || !v_pool || !block_table || !seq_lens || !o) return FA_ERR_INVALID_ARG;
+  if (S < 1 || H < 1 || max_blocks_per_seq < 1 || num_blocks < 1) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(S) * H > INT_MAX / 4) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_blocks_per_seq) * fa::kPage > INT_MAX) return FA_ERR_INVALID_ARG;
+  float sc;
+  if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o))
+    return FA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  const size_t need = fa_decode_workspace_size(S, H, d, max_blocks_per_seq);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
+  const size_t o_bytes = static_cast<size_t>(S) * H * d * (o_dtype == FA_OUT_F32 ? 4 : 2);
+  if (overlaps(o, o_bytes, workspace, need) || (lse && overlaps(lse, static_cast<size_t>(S) * H * 4, workspace, need)))
+    return FA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+
+  fa::DecodeParams p;
+  p.q = static_cast<const uint16_t *>(q);
+  p.kp = static_cast<const uint16_t *>(k_pool);
+  p.vp = static_cast<const uint16_t *>(v_pool);
+  p.table = block_table;
+  p.lens = seq_lens;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.H = H;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.ws = static_cast<float *>(workspace);
+  p.n_split = decode_splits(max_blocks_per_seq);
+  p.o = o;
+  p.o_f32 = o_dtype == FA_OUT_F32;
+  p.lse = lse;
+  p.SH = S * H;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid1(p.n_split, H, S);
+  const int grid2 = (p.SH + 3) / 4;
+  if (d == 128) {
+    fa::fa_decode_partial_kernel<128><<<grid1, fa::kDecodeThreads, 0, s>>>(p);
+    fa::fa_decode_combine_kernel<128><<<grid2, 128, 0, s>>>(p);
+  } else {
+    fa::fa_decode_partial_kernel<64><<<grid1, fa::kDecodeThreads, 0, s>>>(p);
+    fa::fa_decode_combine_kernel<64><<<grid2, 128, 0, s>>>(p);
+  }
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : launch_failed(e);
+}
+
+fa_status fa_get_device_status(fa_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return launch_failed(e);
+  int v = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof v)) != cudaSuccess)
+    return launch_failed(e);
+  if (v != 0) {
+    const int zero = 0;
+    if ((e = cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof zero)) != cudaSuccess)
+      return launch_failed(e);
+  }
+  return static_cast<fa_status>(v);
+}
+
+const char *fa_status_string(fa_status status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: an argument is out of range";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: head dim must be 64 or 128 on an sm_100 GPU";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT: tensors must be 16-byte aligned";
+    case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH: the CUDA launch failed (see fa_last_error_string)";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a kernel abandoned a device-side wait";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: decode workspace missing or too small";
+  }
+  return "unknown fa_status";
+}
+
+const char *fa_last_error_string(void) { return t_last_error.c_str(); }
+
+int fa_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,136 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa_b200.so).
+ *
+ * Operation.  Exact scaled-dot-product attention, forward only:
+ *     O = softmax(scale * Q K^T [+ causal mask]) V,   LSE_i = log sum_j exp(scale * q_i . k_j)
+ * computed tile by tile with a running row max and row sum, so the N x N score matrix never
+ * leaves the chip ("Flash Attention" (velog.io/@myungum), section 2 and its pseudocode: blocks of
+ * Q, K, V are loaded into on-chip memory, the row max m and row sum l are carried across key
+ * blocks, and only O, l, m are written back; "How Flash Attention reduces memory traffic"
+ * (zimaspace), tiling and online softmax).  Work is split over batch, head and query tile
+ * ("FlashAttention-2 GPU work partitioning", section 3).  The paged decode entry point reads its
+ * keys and values through a block table that maps each sequence's logical KV blocks to physical
+ * blocks of a shared pool ("LLM study notes" (devocean.sk.com), paged attention).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never allocates,
+ *     frees or synchronises device memory (except fa_get_device_status, which synchronises the
+ *     given stream).  Every launch is asynchronous on the caller's stream.
+ *   - bf16 inputs (IEEE bfloat16 bit patterns), fp32 accumulation.
+ *   - Arguments are checked on the host before anything is launched; on error nothing runs and a
+ *     status code is returned.  No entry point aborts, traps or prints.
+ *   - Device-side waits are bounded: a kernel that stops making progress records FA_ERR_TIMEOUT in
+ *     a device status word and returns; fa_get_device_status reports and clears it.
+ *   - Thread safety: calls on different streams may run concurrently; the status word is shared.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fa_stream_t; /* the same handle as cudaStream_t; NULL = legacy default */
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1, /* a size, pointer or scale is out of range                         */
+    FA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128, or a non-B200 device        */
+    FA_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned                                  */
+    FA_ERR_LAUNCH = 4,      /* the CUDA launch failed; fa_last_error_string() has the CUDA text  */
+    FA_ERR_TIMEOUT = 5,     /* a kernel gave up waiting (reported by fa_get_device_status)       */
+    FA_ERR_WORKSPACE = 6    /* the decode workspace is NULL or smaller than required             */
+} fa_status;
+
+typedef enum {
+    FA_OUT_BF16 = 0, /* O written as bf16 (round to nearest even) */
+    FA_OUT_F32 = 1   /* O written as fp32                          */
+} fa_out_dtype;
+
+/*
+ * fa_fwd -- prefill / full-sequence attention forward.
+ *
+ * Defined by the plain attention of "LLM study notes", self-attention steps (dot product of query
+ * and key, divide by sqrt(d_k), softmax, weight the values), evaluated with the tiled online
+ * softmax of "Flash Attention" (myungum), section 2.  Causal: query i sees keys 0..i
+ * ("FlashAttention-2 GPU work partitioning", section 4).
+ *
+ *   q, k, v   bf16 [B, H, N, d], contiguous (row i of head (b,h) at ((b*H + h)*N + i)*d).
+ *             May alias one another.  16-byte aligned.
+ *   o         [B, H, N, d] contiguous, bf16 or fp32 per o_dtype.  16-byte aligned.  Must not
+ *             overlap q, k, v or lse.
+ *   lse       fp32 [B, H, N] (natural log of the row sum of exp(scaled scores)), or NULL.
+ *   B, H, N   >= 1;  B*H*N*d must fit in int64;  B*H < 2^31;  N < 2^31.
+ *   d         64 or 128 (else FA_ERR_UNSUPPORTED).
+ *   causal    0 or 1.
+ *   scale     > 0 and finite; pass 0 (or any value <= 0) for 1/sqrt(d).  NaN/inf -> INVALID_ARG.
+ *   stream    the stream to launch on.
+ * Returns FA_OK once the kernel is queued.
+ */
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, fa_out_dtype o_dtype,
+                 float *lse, int B, int H, int N, int d, int causal, float scale,
+                 fa_stream_t stream);
+
+/*
+ * fa_decode_workspace_size -- bytes of device workspace fa_decode_paged needs for these sizes.
+ * The split of each sequence's context into chunks depends only on the arguments here, so the
+ * same values must be passed to fa_decode_paged.  Returns 0 on invalid sizes.
+ */
+size_t fa_decode_workspace_size(int num_seqs, int H, int d, int max_blocks_per_seq);
+
+/*
+ * fa_decode_paged -- one decode step (query length 1) over a paged KV cache.
+ *
+ * The cache is a pool of fixed 16-token blocks; sequence s's logical block t lives in physical
+ * block block_table[s * max_blocks_per_seq + t] ("LLM study notes", paged attention: the block
+ * table makes logically contiguous KV memory out of physically scattered blocks).  The query of
+ * sequence s attends to its seq_lens[s] cached tokens (it sits after them, so nothing is masked).
+ * The context is split into chunks processed in parallel; the per-chunk running max, sum and
+ * unnormalised output are merged with the same rescaling rule the tiled algorithm uses between
+ * key blocks ("Flash Attention" (myungum), section 2, the m_new / l_new update).
+ *
+ *   q            bf16 [S, H, d] contiguous.
+ *   k_pool,
+ *   v_pool       bf16 [num_blocks, H, 16, d] contiguous (one 16 x d block per (block, head)).
+ *   block_table  int32 [S, max_blocks_per_seq], device; entries t < ceil(seq_lens[s]/16) must be
+ *                in [0, num_blocks); later entries are never read.
+ *   seq_lens     int32 [S], device; each in [1, 16 * max_blocks_per_seq].  Values are not
+ *                checked on the host (they live on the device); out-of-range lengths are clamped
+ *                to that interval by the kernel.
+ *   o            [S, H, d], bf16 or fp32 per o_dtype;  lse: fp32 [S, H] or NULL.
+ *   S, H         >= 1;  d: 64 or 128;  scale as for fa_fwd.
+ *   workspace    device scratch of at least fa_decode_workspace_size(S, H, d, max_blocks_per_seq)
+ *                bytes, 16-byte aligned, owned by the caller; its contents need no initialisation
+ *                and are garbage afterwards.  Two calls in flight at once need separate workspaces.
+ * Returns FA_OK once the kernels are queued.
+ */
+fa_status fa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
+                          const int32_t *block_table, int max_blocks_per_seq,
+                          const int32_t *seq_lens, int num_blocks, void *o, fa_out_dtype o_dtype,
+                          float *lse, int S, int H, int d, float scale, void *workspace,
+                          size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fa_get_device_status -- synchronises `stream`, then reads and clears the library's device
+ * status word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel abandoned a wait), or FA_ERR_LAUNCH if the
+ * synchronisation itself reported a CUDA error.
+ */
+fa_status fa_get_device_status(fa_stream_t stream);
+
+/* Static text for a status code. */
+const char *fa_status_string(fa_status status);
+
+/* The CUDA error text of the last FA_ERR_LAUNCH on this thread ("" if none). */
+const char *fa_last_error_string(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,69 @@
+"""Helpers for the GPU-vs-oracle parity tests: inputs from the shared generator, outputs compared
+element by element with the tolerance the acceptance bar states
+(max|dO| <= 1e-2, mean|dO| <= 1e-3, max|dLSE| <= 1e-3)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import workloads as W
+from oracle import oracle as orc
+
+TOL_MAX_O = 1e-2
+TOL_MEAN_O = 1e-3
+TOL_LSE = 1e-3
+
+
+def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+    o_gpu = np.asarray(o_gpu, np.float64)
+    d = np.abs(o_gpu - o_ref)
+    assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite output"
+    mx, mean = float(d.max()), float(d.mean())
+    assert mx <= TOL_MAX_O, f"{what}: max|dO| {mx:.3e} > {TOL_MAX_O}"
+    assert mean <= TOL_MEAN_O, f"{what}: mean|dO| {mean:.3e} > {TOL_MEAN_O}"
+    if lse_gpu is not None:
+        dl = float(np.abs(np.asarray(lse_gpu, np.float64) - lse_ref).max())
+        assert dl <= TOL_LSE, f"{what}: max|dLSE| {dl:.3e} > {TOL_LSE}"
+    return mx, mean
+
+
+def sample_rows(case: W.PrefillCase, n_heads: int = 6, n_random: int = 24, seed: int = 1):
+    """(bh, row) pairs: a spread of heads; per head rows 0, 127, 128, N-1, every 128-row tile
+    boundary (up to 16 of them) and seeded random rows."""
+    rng = np.random.default_rng(seed)
+    BH, N = case.B * case.H, case.N
+    heads = sorted(set([0, BH - 1] + list(rng.integers(0, BH, n_heads))))
+    pairs = []
+    for bh in heads:
+        rows = {0, min(127, N - 1), min(128, N - 1), N - 1}
+        bounds = list(range(0, N, 128))
+        step = max(1, len(bounds) // 16)
+        for b in bounds[::step]:
+            rows.update({b, max(0, b - 1)})
+        rows.update(int(r) for r in rng.integers(0, N, n_random))
+        pairs += [(bh, r) for r in sorted(rows)]
+    return np.array(pairs, dtype=np.int64)
+
+
+def run_prefill(case: W.PrefillCase, out_dtype=torch.float32, full: bool | None = None):
+    """Run fa_fwd on the case and compare with the oracle (all rows if small, else sampled)."""
+    import exact_attention_158_b200 as fa
+    q, k, v = W.make_prefill(case, device="cuda")
+    o, lse = fa.fa_fwd(q, k, v, causal=case.causal, scale=case.scale, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    qb, kb, vb = (W.bf16_bits(t) for t in (q, k, v))
+    BH, N, d = case.B * case.H, case.N, case.d
+    if full is None:
+        full = BH * N * N * d <= 3e9
+    if full:
+        o_ref, lse_ref = orc.attention(qb.reshape(BH, N, d), kb.reshape(BH, N, d),
+                                       vb.reshape(BH, N, d), case.causal, case.scale)
+        return assert_close(o.float().cpu().numpy().reshape(BH, N, d), lse.cpu().numpy().reshape(BH, N),
+                            o_ref, lse_ref, case.name)
+    pairs = sample_rows(case)
+    o_ref, lse_ref = orc.attention_rows(qb.reshape(BH, N, d), kb.reshape(BH, N, d),
+                                        vb.reshape(BH, N, d), case.causal, case.scale, pairs)
+    og = o.float().reshape(BH, N, d)[pairs[:, 0], pairs[:, 1]].cpu().numpy()
+    lg = lse.reshape(BH, N)[pairs[:, 0], pairs[:, 1]].cpu().numpy()
+    return assert_close(og, lg, o_ref, lse_ref, case.name + " (sampled rows)")

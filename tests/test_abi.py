@@ -1,0 +1,89 @@
+"""The C-ABI library: it loads, exports every symbol include/fa.h declares, and its host-side
+argument checks reject bad calls before anything is launched (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_158_b200 as fa
+from exact_attention_158_b200 import build as fab
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fab.build()
+    return fa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_functions() == sorted(fa.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} missing from {fa.library_path()}"
+
+
+def test_status_strings_and_version(lib):
+    for code, name in fa.STATUS.items():
+        assert lib.fa_status_string(code).decode().startswith(name)
+    assert lib.fa_version() >= 100
+
+
+# fake device addresses: never dereferenced, every call below fails its host-side checks first
+A = 1 << 20
+
+
+def fwd(lib, q=A, k=2 * A, v=3 * A, o=4 * A, dt=0, lse=None, B=1, H=1, N=8, d=64, causal=0,
+        scale=0.0):
+    return lib.fa_fwd(q, k, v, o, dt, lse, B, H, N, d, causal, scale, None)
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert fwd(lib, q=None) == 1
+    assert fwd(lib, B=0) == 1 and fwd(lib, H=0) == 1 and fwd(lib, N=0) == 1
+    assert fwd(lib, causal=2) == 1
+    assert fwd(lib, dt=7) == 1
+    assert fwd(lib, d=96) == 2 and fwd(lib, d=256) == 2
+    assert fwd(lib, scale=float("nan")) == 1 and fwd(lib, scale=float("inf")) == 1
+    assert fwd(lib, q=A + 8) == 3 and fwd(lib, o=4 * A + 4) == 3
+    assert fwd(lib, lse=5 * A + 2) == 3
+    # output overlapping an input
+    assert fwd(lib, o=A + 16) == 1
+    assert fwd(lib, lse=2 * A + 64) == 1
+
+
+def dec(lib, ws=8 * A, ws_bytes=1 << 30, S=2, H=2, d=128, maxb=4, P=8, table=5 * A, lens=6 * A,
+        q=A, o=7 * A, lse=None):
+    return lib.fa_decode_paged(q, 2 * A, 3 * A, table, maxb, lens, P, o, 0, lse, S, H, d, 0.0, ws,
+                               ws_bytes, None)
+
+
+def test_decode_workspace_and_rejections(lib):
+    need = lib.fa_decode_workspace_size(64, 32, 128, 512)
+    assert need == 64 * 32 * 16 * (128 + 2) * 4  # 512 blocks -> 16 chunks of 32 blocks
+    assert lib.fa_decode_workspace_size(0, 32, 128, 512) == 0
+    assert lib.fa_decode_workspace_size(1, 1, 96, 1) == 0
+    assert dec(lib, ws=None) == 6
+    assert dec(lib, ws_bytes=16) == 6
+    assert dec(lib, S=0) == 1 and dec(lib, maxb=0) == 1 and dec(lib, P=0) == 1
+    assert dec(lib, d=80) == 2
+    assert dec(lib, table=5 * A + 2) == 3
+    assert dec(lib, ws=8 * A + 8) == 3
+    assert dec(lib, o=8 * A) == 1  # output overlaps the workspace
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.fa_fwd(x, x, x)

@@ -1,0 +1,86 @@
+"""fa_fwd (tcgen05 prefill kernel) against the fp64 oracle on the same seeded bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_tiny(causal, out_dtype):
+    parity.run_prefill(W.PrefillCase("tiny", 1, 1, 256, 64, causal), out_dtype, full=True)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 2, 127, 128, 129, 255, 256, 257, 383, 1000])
+def test_ragged_lengths(N, causal, d):
+    parity.run_prefill(W.PrefillCase(f"ragged_N{N}", 2, 2, N, d, causal), torch.float32, full=True)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_multi_tile_full(causal):
+    # several heads, 8 query pairs, 16 key blocks: exercises the ring, the persistent loop and
+    # the causal pairing of work units, every row checked
+    parity.run_prefill(W.PrefillCase("multi", 2, 3, 2048, 128, causal), torch.float32, full=True)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_prefill_config(causal, out_dtype):
+    # B=8, H=16, N=2048, d=128: the launch configuration the bench times; sampled rows
+    parity.run_prefill(W.PrefillCase("prefill", 8, 16, 2048, 128, causal), out_dtype)
+
+
+@pytest.mark.parametrize("case", W.sweep_cases(128) + W.sweep_cases(64),
+                         ids=lambda c: f"{c.name}_N{c.N}_{'causal' if c.causal else 'full'}")
+def test_sweep(case):
+    parity.run_prefill(case, torch.bfloat16)
+
+
+def test_peaked_rows_full_small():
+    # 1% of key rows scaled x8 gives peaked softmax rows: full check on a small shape
+    parity.run_prefill(W.PrefillCase("peaked", 2, 4, 1024, 64, True, peaked=True), torch.float32,
+                       full=True)
+
+
+def test_scale_override_and_aliasing():
+    import exact_attention_158_b200 as fa
+    from oracle import oracle as orc
+    case = W.PrefillCase("alias", 1, 2, 300, 128, False)
+    q, _, _ = W.make_prefill(case, device="cuda")
+    o, lse = fa.fa_fwd(q, q, q, causal=False, scale=0.05, out_dtype=torch.float32)
+    qb = W.bf16_bits(q).reshape(2, 300, 128)
+    o_ref, lse_ref = orc.attention(qb, qb, qb, False, 0.05)
+    parity.assert_close(o.cpu().numpy().reshape(2, 300, 128), lse.cpu().numpy().reshape(2, 300),
+                        o_ref, lse_ref, "q=k=v, scale 0.05")
+
+
+def test_guard_bytes_untouched():
+    import exact_attention_158_b200 as fa
+    case = W.PrefillCase("guard", 1, 3, 200, 64, True)
+    q, k, v = W.make_prefill(case, device="cuda")
+    n = 3 * 200 * 64
+    pad = 4096
+    buf = torch.full((n + 2 * pad,), float("nan"), dtype=torch.float32, device="cuda")
+    lbuf = torch.full((3 * 200 + 2 * pad,), float("nan"), dtype=torch.float32, device="cuda")
+    o = buf[pad:pad + n].view(1, 3, 200, 64)
+    lse = lbuf[pad:pad + 600].view(1, 3, 200)
+    fa.fa_fwd(q, k, v, causal=True, out_dtype=torch.float32, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.isnan(buf[:pad]).all() and torch.isnan(buf[pad + n:]).all()
+    assert torch.isnan(lbuf[:pad]).all() and torch.isnan(lbuf[pad + 600:]).all()
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+def test_repeatable_bitwise():
+    import exact_attention_158_b200 as fa
+    case = W.PrefillCase("rep", 2, 4, 1024, 128, True)
+    q, k, v = W.make_prefill(case, device="cuda")
+    o1, l1 = fa.fa_fwd(q, k, v, causal=True)
+    o2, l2 = fa.fa_fwd(q, k, v, causal=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
