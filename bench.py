@@ -1,0 +1,434 @@
+"""Throughput of the exact-attention hot path on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...
+
+A step is one pass of the whole prefill hot path over the workload "prefill B8 H16 N2048 d128"
+(bf16 Q/K/V i.i.d. N(0,1), seeded): one non-causal and one causal fa_fwd launch (tile scheduler,
+TMA loads, Q K^T, mask, online softmax, rescale, P V and epilogue all run inside them).
+`value` is attention TFLOP/s (4 B H N^2 d per non-causal pass, half that causal) over all ranks;
+the L2 is flushed (a 256 MiB write) before every timed step and the flush is outside the timed
+events.  With N ranks each rank runs the same independent (b, h) workload (weak scaling; heads are
+independent, so there is no collective on the data path).
+
+Extra keys: `roofline` (prefill kernel vs the measured dense bf16 peak), `cpu_baseline` (the fp64
+oracle on this host's cores, a bounded row sample), `e2e` (the same metric through the Python API
+with Q/K/V copied from pinned host memory and O/LSE copied back inside the timed region), `sweep`
+(the sequence-length grid, d = 128 and d = 64), `decode` (paged decode GB/s vs HBM) and `clocks`.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16 peak) vs seqlen; decode GB/s"
+UNIT = "TFLOP/s"
+WORKLOAD = "prefill B8 H16 N2048 d128, causal + non-causal"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+KERNEL_SOURCES = ["exact_attention_158_b200/csrc/fa_prefill.cuh",
+                  "exact_attention_158_b200/csrc/sm100_ptx.cuh"]
+DECODE_SOURCES = ["exact_attention_158_b200/csrc/fa_decode.cuh",
+                  "exact_attention_158_b200/csrc/sm100_ptx.cuh"]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    return dict(FALLBACK_PEAKS)
+
+
+def source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(name: str, paths):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f).get(name)
+    if not t or t.get("source_hash") != source_hash(paths):
+        return None
+    return t.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no clocks rather than guess
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------------
+# timing helpers
+# ---------------------------------------------------------------------------------------------
+class Flusher:
+    def __init__(self, device):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def time_launches(fn, steps, warmup, flush, stream):
+    """Run fn() warmup times, then `steps` times with an L2 flush before each; returns the list of
+    per-step device times (ms) from CUDA events recorded on `stream`."""
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def dist_max(x: float) -> float:
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+    return x
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on this host's cores, bounded sample of rows
+# ---------------------------------------------------------------------------------------------
+_CPU_INPUTS = None
+
+
+def cpu_baseline(target_s: float = 12.0):
+    import numpy as np
+    from oracle import oracle as orc
+    global _CPU_INPUTS
+    BH, N, d = 8 * 16, 2048, 128
+    if _CPU_INPUTS is None:
+        q, k, v = W.make_prefill(W.prefill_cases()[0], device="cpu")
+        _CPU_INPUTS = tuple(W.bf16_bits(t).reshape(BH, N, d) for t in (q, k, v))
+    qb, kb, vb = _CPU_INPUTS
+    threads = orc.default_threads()
+    rng = np.random.default_rng(0)
+    flops = 0.0
+    rows = 0
+    t0 = time.perf_counter()
+    batch = max(64, threads * 16)
+    while time.perf_counter() - t0 < target_s:
+        for causal in (False, True):
+            pairs = np.stack([rng.integers(0, BH, batch), rng.integers(0, N, batch)], 1)
+            orc.attention_rows(qb, kb, vb, causal, 1 / math.sqrt(d), pairs, threads)
+            # exact FLOPs of these rows: 4 d per visible key
+            vis = (pairs[:, 1] + 1) if causal else np.full(batch, N)
+            flops += float(4.0 * d * vis.sum())
+            rows += batch
+    el = time.perf_counter() - t0
+    return {"value": flops / el / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} query rows of {WORKLOAD} (half causal), fp64, {el:.1f} s; "
+                      "throughput scaled by the exact FLOPs of the sampled rows"}
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+def run_prefill_case(fa, case, steps, warmup, flush, stream, out_dtype=torch.bfloat16):
+    q, k, v = W.make_prefill(case, device="cuda")
+    o = torch.empty_like(q) if out_dtype == torch.bfloat16 else torch.empty(q.shape, dtype=out_dtype, device="cuda")
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    fn = lambda: fa.fa_fwd(q, k, v, causal=case.causal, scale=case.scale, out=o, lse=lse,
+                           out_dtype=out_dtype)
+    ts = time_launches(fn, steps, warmup, flush, stream)
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during the bench")
+    return ts
+
+
+def bench_decode(fa, args, dev, flush, stream, pk):
+    case = W.DecodeCase("decode")
+    inp = W.make_decode(case, device=dev)
+    o = torch.empty_like(inp["q"])
+    lse = torch.empty(inp["q"].shape[:2], dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_decode_workspace_size(case.S, case.H, case.d, inp["max_blocks"]),
+                     dtype=torch.uint8, device=dev)
+    fn = lambda: fa.fa_decode_paged(inp["q"], inp["k_pool"], inp["v_pool"], inp["block_table"],
+                                    inp["seq_lens"], scale=case.scale, out=o, lse=lse,
+                                    workspace=ws)
+    torch.cuda.nvtx.range_push("bench_decode_timed")
+    ts = time_launches(fn, args.sweep_steps, 3, flush, stream)
+    torch.cuda.nvtx.range_pop()
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during the decode bench")
+    ms = statistics.median(ts)
+    nbytes = W.decode_bytes(inp["lens"], case.H, case.d, inp["max_blocks"])
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"metric": "paged decode GB/s", "workload": "64 seqs, q len 1, H32 d128, "
+            "context U[512,8192], 16-token pages, permuted block table",
+            "ms": round(ms, 4), "value": round(gbs, 1), "unit": "GB/s",
+            "algorithmic_bytes": nbytes, "tokens": sum(inp["lens"]),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "traffic": committed_traffic("decode", DECODE_SOURCES)},
+            "launches_per_step": 2}
+
+
+def bench_ours(args, rank, world):
+    import exact_attention_158_b200 as fa
+    fa.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    flush = Flusher(dev)
+    pk = peaks()
+    if args.only == "decode":
+        return {"metric": METRIC, "decode": bench_decode(fa, args, dev, flush, stream, pk)}
+
+    # ---- headline: prefill config, non-causal + causal per step
+    cases = W.prefill_cases()
+    inputs = [W.make_prefill(c, device=dev) for c in cases]
+    outs = [(torch.empty_like(q), torch.empty(q.shape[:3], dtype=torch.float32, device=dev))
+            for q, _, _ in inputs]
+    kernel_ms = {False: [], True: []}
+
+    def step():
+        for c, (q, k, v), (o, lse) in zip(cases, inputs, outs):
+            fa.fa_fwd(q, k, v, causal=c.causal, scale=c.scale, out=o, lse=lse)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in cases] for _ in range(args.steps)]
+    torch.cuda.nvtx.range_push("bench_timed")
+    with ClockSampler(dev.index) as clk:
+        for st in range(args.steps):
+            flush()
+            for ci, (c, (q, k, v), (o, lse)) in enumerate(zip(cases, inputs, outs)):
+                a, b = evs[st][ci]
+                a.record(stream)
+                fa.fa_fwd(q, k, v, causal=c.causal, scale=c.scale, out=o, lse=lse)
+                b.record(stream)
+        torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    barrier()
+    torch.cuda.synchronize()
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during the timed region")
+    for st in range(args.steps):
+        for ci, c in enumerate(cases):
+            kernel_ms[c.causal].append(evs[st][ci][0].elapsed_time(evs[st][ci][1]))
+    step_ms = statistics.mean(kernel_ms[False]) + statistics.mean(kernel_ms[True])
+    step_ms_max = dist_max(step_ms)
+    flops_step = sum(c.flops for c in cases)
+    value = world * flops_step / (step_ms_max * 1e-3) / 1e12
+    peak_key = "bf16_tflops"
+    achieved = flops_step / (step_ms * 1e-3) / 1e12
+    traffic = committed_traffic("prefill", KERNEL_SOURCES)
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk[peak_key],
+                "unit": "TFLOP/s", "frac": round(achieved / pk[peak_key], 4),
+                "peak_source": f"{pk['source']} {peak_key} (burst: the kernel is timed alone)",
+                "traffic": traffic,
+                "per_variant": {
+                    ("causal" if c else "non_causal"): {
+                        "ms": round(statistics.mean(kernel_ms[c]), 4),
+                        "tflops": round(cases[int(c)].flops / (statistics.mean(kernel_ms[c]) * 1e-3) / 1e12, 1)}
+                    for c in (False, True)}}
+    clocks = clk.summary()
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, counter-based generator)",
+        "config": {"workload": WORKLOAD, "B": 8, "H": 16, "N": 2048, "d": 128,
+                   "causal": "both (one launch each per step)", "o_dtype": "bf16",
+                   "parallelism": f"replicas x{world} (independent heads per GPU)",
+                   "l2": "flushed (256 MiB write) before every timed step, outside the events"},
+        "roofline": roofline, "gpu_launches": 2 * args.steps, "clocks": clocks,
+    }
+    if args.only == "prefill":
+        return result
+
+    # ---- e2e through the Python API with host buffers
+    host_in = [[t.cpu().pin_memory() for t in trio] for trio in inputs]
+    host_out = [(torch.empty(q.shape, dtype=torch.bfloat16).pin_memory(),
+                 torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()) for q, _, _ in inputs]
+    dev_in = [[torch.empty_like(t) for t in trio] for trio in inputs]
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for c, hi, di, (ho, hl) in zip(cases, host_in, dev_in, host_out):
+            for h, d_ in zip(hi, di):
+                d_.copy_(h, non_blocking=True)
+            o, lse = fa.fa_fwd(di[0], di[1], di[2], causal=c.causal, scale=c.scale)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+    e2e_ts = time_launches(e2e_step, e2e_steps, 2, flush, stream)
+    e2e_ms = dist_max(statistics.mean(e2e_ts))
+    h2d = sum(t.numel() * t.element_size() for hi in host_in for t in hi)
+    d2h = sum(o.numel() * o.element_size() + l.numel() * l.element_size() for o, l in host_out)
+    e2e = {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+    del inputs, outs, host_in, host_out, dev_in
+    torch.cuda.empty_cache()
+
+    # ---- sequence-length sweep (the pages' benchmark grid)
+    sweep = []
+    if not args.no_sweep:
+        for d in (128, 64):
+            for case in W.sweep_cases(d):
+                ts = run_prefill_case(fa, case, args.sweep_steps, 3, flush, stream)
+                ms = statistics.median(ts)
+                tf = case.flops / (ms * 1e-3) / 1e12
+                intensity = case.flops / (4 * case.B * case.H * case.N * case.d * 2 + case.B * case.H * case.N * 4)
+                attainable = min(pk["bf16_tflops"], intensity * pk["hbm_gbs"] / 1e3)
+                sweep.append({"d": d, "N": case.N, "B": case.B, "H": case.H, "causal": case.causal,
+                              "ms": round(ms, 4), "tflops": round(tf, 1),
+                              "frac_peak": round(tf / pk["bf16_tflops"], 4),
+                              "frac_attainable": round(tf / attainable, 4)})
+                torch.cuda.empty_cache()
+
+    # ---- paged decode (HBM bound)
+    dec = None if args.no_decode else bench_decode(fa, args, dev, flush, stream, pk)
+
+    result.update({"e2e": e2e, "sweep": sweep, "decode": dec})
+    return result
+
+
+# ---------------------------------------------------------------------------------------------
+def bench_reference(args):
+    """The oracle as it stands, on this host's cores, for the same metric and workload."""
+    steps = []
+    cb = None
+    for _ in range(args.warmup):
+        cpu_baseline(target_s=2.0)
+    for _ in range(args.steps):
+        cb = cpu_baseline(target_s=max(2.0, 20.0 / max(args.steps, 1)))
+        steps.append(cb["value"])
+    value = statistics.mean(steps)
+    cb = dict(cb, value=value)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": 8, "H": 16, "N": 2048, "d": 128},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--sweep-steps", type=int, default=20)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="prefill: the headline loop alone; decode: the decode loop alone")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(bench_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    out = bench_ours(args, rank, world)
+    if rank == 0 and world == 1 and args.only == "all" and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline()
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()
