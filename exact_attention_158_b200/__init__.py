@@ -17,7 +17,8 @@ import torch
 
 from . import build as _build
 
-__all__ = ["fa_fwd", "fa_decode_paged", "fa_decode_workspace_size", "device_status",
+__all__ = ["fa_fwd", "fa_decode_paged", "fa_decode_paged_noalloc", "fa_decode_workspace_size",
+           "NOALLOC_SCRATCH_BYTES", "device_status",
            "FaError", "library_path", "load_library", "EXPORTED_SYMBOLS", "STATUS"]
 
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_ALIGNMENT",
@@ -25,8 +26,8 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 FA_OUT_BF16, FA_OUT_F32 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
-                    "fa_get_device_status", "fa_status_string", "fa_last_error_string",
-                    "fa_version")
+                    "fa_decode_paged_noalloc", "fa_get_device_status", "fa_status_string",
+                    "fa_last_error_string", "fa_version")
 
 _lib = None
 
@@ -181,3 +182,33 @@ def fa_decode_paged(q, k_pool, v_pool, block_table, seq_lens, scale: float | Non
 def device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the library's device status word."""
     return int(load_library().fa_get_device_status(_stream_handle(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # FA_NOALLOC_SCRATCH_BYTES in include/fa.h
+
+
+def fa_decode_paged_noalloc(q, k_pool, v_pool, block_table, seq_lens, out, lse=None,
+                            scale: float | None = None, stream=None):
+    """fa_decode_paged for callers that cannot allocate device memory at decode time.
+
+    The caller passes every buffer, ``out`` included (bf16 or fp32 [S, H, d]; ``lse`` fp32
+    [S, H] or None); the split-context scratch is the library's static 32 MiB device array, so
+    nothing is allocated here or in the library.  Calls that overlap on the GPU share that array
+    and race: serialise them.  Sizes needing more scratch than the array holds raise FaError."""
+    lib = load_library()
+    f = lib.fa_decode_paged_noalloc
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, i32, vp, i32, i32, i32, ctypes.c_float, vp]
+    f.restype = i32
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _require(t, n)
+    _require(block_table, "block_table", torch.int32)
+    _require(seq_lens, "seq_lens", torch.int32)
+    _require(out, "out", out.dtype)
+    S, H, d = q.shape
+    st = f(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),
+           block_table.shape[1], seq_lens.data_ptr(), k_pool.shape[0], out.data_ptr(),
+           _out_code(out.dtype), lse.data_ptr() if lse is not None else None, S, H, d,
+           float(scale) if scale is not None else 0.0, _stream_handle(stream))
+    _check(st, "fa_decode_paged_noalloc")
+    return out, lse

@@ -249,6 +249,103 @@ fa_status fa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
   return e == cudaSuccess ? FA_OK : launch_failed(e);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free decode: the split-context scratch lives in a static device array.
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+// Held by every GPU that loads this library, for the life of the process.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on `dev` (the current device), looked up once per device.
+// In host code the array's name is only a host-side stand-in, never a device address.
+fa_status noalloc_scratch(int dev, void **out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return launch_failed(e);
+    if (!ptr) {
+      t_last_error = "cudaGetSymbolAddress returned no address for the decode scratch";
+      return FA_ERR_LAUNCH;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_decode_paged_noalloc(const void *q, const void *k_pool, const void *v_pool,
+                                  const int32_t *block_table, int max_blocks_per_seq,
+                                  const int32_t *seq_lens, int num_blocks, void *o,
+                                  fa_out_dtype o_dtype, float *lse, int S, int H, int d,
+                                  float scale, fa_stream_t stream) {
+  if (!q || !k_pool || !v_pool || !block_table || !seq_lens || !o) return FA_ERR_INVALID_ARG;
+  if (S < 1 || H < 1 || max_blocks_per_seq < 1 || num_blocks < 1) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(S) * H > INT_MAX / 4) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_blocks_per_seq) * fa::kPage > INT_MAX) return FA_ERR_INVALID_ARG;
+  float sc;
+  if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o))
+    return FA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  const size_t need = fa_decode_workspace_size(S, H, d, max_blocks_per_seq);
+  if (need > FA_NOALLOC_SCRATCH_BYTES) {
+    t_last_error = "fa_decode_paged_noalloc: these sizes need " + std::to_string(need) +
+                   " bytes of scratch; the static array holds " +
+                   std::to_string(FA_NOALLOC_SCRATCH_BYTES);
+    return FA_ERR_WORKSPACE;
+  }
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(dev_id, &scratch)) != FA_OK) return st;
+
+  fa::DecodeParams p;
+  p.q = static_cast<const uint16_t *>(q);
+  p.kp = static_cast<const uint16_t *>(k_pool);
+  p.vp = static_cast<const uint16_t *>(v_pool);
+  p.table = block_table;
+  p.lens = seq_lens;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.H = H;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.ws = static_cast<float *>(scratch);
+  p.n_split = decode_splits(max_blocks_per_seq);
+  p.o = o;
+  p.o_f32 = o_dtype == FA_OUT_F32;
+  p.lse = lse;
+  p.SH = S * H;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid1(p.n_split, H, S);
+  const int grid2 = (p.SH + 3) / 4;
+  if (d == 128) {
+    fa::fa_decode_partial_kernel<128><<<grid1, fa::kDecodeThreads, 0, s>>>(p);
+    fa::fa_decode_combine_kernel<128><<<grid2, 128, 0, s>>>(p);
+  } else {
+    fa::fa_decode_partial_kernel<64><<<grid1, fa::kDecodeThreads, 0, s>>>(p);
+    fa::fa_decode_combine_kernel<64><<<grid2, 128, 0, s>>>(p);
+  }
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : launch_failed(e);
+}
+
 fa_status fa_get_device_status(fa_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return launch_failed(e);

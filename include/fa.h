@@ -114,6 +114,35 @@ fa_status fa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
                           size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_decode_paged_noalloc -- fa_decode_paged without a caller-supplied workspace and without any
+ * allocation.  No counterpart in the paper: this is a deployment variant of the same decode step,
+ * not part of the method.
+ *
+ * Who needs it: callers that cannot call cudaMalloc at decode time -- for instance a serving
+ * engine that has handed almost all device memory to its own KV-cache pool and allocator (a
+ * cudaMalloc would fail or fragment that pool), or a decode loop that cannot afford the
+ * device-wide synchronisation and latency that cudaMalloc/cudaFree may cost.  Such callers still
+ * own q, the pools, the table, the lengths, o and lse; only the split-context scratch moves.
+ *
+ * The scratch is a static device array of FA_NOALLOC_SCRATCH_BYTES inside this library: every
+ * GPU that loads the library holds it until the process exits.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress, no allocation); make that first call
+ * before any stream capture.  Arguments are as for fa_decode_paged; sizes whose
+ * fa_decode_workspace_size(S, H, d, max_blocks_per_seq) exceeds FA_NOALLOC_SCRATCH_BYTES return
+ * FA_ERR_WORKSPACE (fa_last_error_string() says how many bytes were needed) and launch nothing.
+ * No slot of the array needs to start at zero: every slot a call reads was written earlier in
+ * that same call.  All calls share the one array, so two calls that overlap on the GPU (other
+ * streams, other host threads) race and corrupt each other's results: serialise them.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+fa_status fa_decode_paged_noalloc(const void *q, const void *k_pool, const void *v_pool,
+                                  const int32_t *block_table, int max_blocks_per_seq,
+                                  const int32_t *seq_lens, int num_blocks, void *o,
+                                  fa_out_dtype o_dtype, float *lse, int S, int H, int d,
+                                  float scale, fa_stream_t stream);
+
+/*
  * fa_get_device_status -- synchronises `stream`, then reads and clears the library's device
  * status word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel abandoned a wait), or FA_ERR_LAUNCH if the
  * synchronisation itself reported a CUDA error.
@@ -123,7 +152,8 @@ fa_status fa_get_device_status(fa_stream_t stream);
 /* Static text for a status code. */
 const char *fa_status_string(fa_status status);
 
-/* The CUDA error text of the last FA_ERR_LAUNCH on this thread ("" if none). */
+/* The CUDA error text of the last FA_ERR_LAUNCH on this thread, or the scratch size that
+ * fa_decode_paged_noalloc needed when it returned FA_ERR_WORKSPACE ("" if none). */
 const char *fa_last_error_string(void);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
