@@ -125,7 +125,7 @@ fa_status launch_prefill(DeviceInfo &dev, const void *q, const void *k, const vo
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.num_pairs = (N + 2 * fa::kBM - 1) / (2 * fa::kBM);
-  p.num_super = causal ? BH * ((p.num_pairs + 1) / 2) : BH * p.num_pairs;
+  p.num_units = BH * p.num_pairs;
   const int slot = HD == 128 ? 1 : 0;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
@@ -137,7 +137,7 @@ fa_status launch_prefill(DeviceInfo &dev, const void *q, const void *k, const vo
       dev.prefill_attr[slot] = true;
     }
   }
-  const int grid = p.num_super < dev.num_sms ? p.num_super : dev.num_sms;
+  const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
   fa::fa_prefill_kernel<HD><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : launch_failed(e);

@@ -30,6 +30,17 @@ constexpr int kBN = 128;  // keys per key/value block
 constexpr int kPrefillThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale: tolerate a stale max up to 2^8 below
 constexpr float kLn2 = 0.6931471805599453f;
+#ifndef FA_POLY_EVERY
+#define FA_POLY_EVERY 0
+#endif
+#ifndef FA_OPTIMISTIC_EXP
+#define FA_OPTIMISTIC_EXP 0
+#endif
+#ifndef FA_KV_STAGES_D128
+#define FA_KV_STAGES_D128 4
+#endif
+// every FA_POLY_EVERY-th pair of P's exponentials on the FMA pipe, the rest on MUFU (0: all MUFU)
+constexpr int kPolyEvery = FA_POLY_EVERY;
 
 template <int HD>
 struct PrefillCfg {
@@ -37,7 +48,7 @@ struct PrefillCfg {
   static constexpr int kChunks = HD / 64;          // 64-element (128-byte) swizzle chunks per row
   static constexpr int kChunkBytes = 128 * 128;    // 128 rows x 128 bytes
   static constexpr int kTileBytes = 128 * HD * 2;  // one 128 x HD bf16 tile
-  static constexpr int kStages = HD == 128 ? 4 : 8;
+  static constexpr int kStages = HD == 128 ? FA_KV_STAGES_D128 : 8;
   static constexpr int kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + HD;
   static constexpr int kNumBars = 1 + 1 + 2 * kStages + 2 + 2 + 2 + 1;
@@ -54,34 +65,36 @@ struct PrefillParams {
   int BH, N, causal;
   float scale_log2;  // scale * log2(e)
   int num_pairs;     // ceil(N / 256)
-  int num_super;     // work units handed out round-robin to the persistent CTAs
+  int num_units;     // BH * num_pairs query-tile pairs, scheduled over the persistent CTAs
 };
 
-// A work unit ("super tile") is one or two query-tile pairs of one (b, h).  Causal units pair the
-// query pair p with the pair num_pairs-1-p, whose key-block counts add up to a constant, so every
-// unit costs the same; non-causal units are single pairs.  Units are numbered head-major so CTAs
-// running at the same time share the same heads' K/V in L2.
+// Work units are query-tile pairs (two 128-row tiles of one (b, h) that share every K/V block).
+// Non-causal units all cost the same; they are numbered head-major (unit = bh * pairs + pair) so
+// the CTAs running at the same time share a few heads' K/V in L2, and handed out round-robin.
+// Causal units cost in proportion to their key-block count (4p + 3 blocks for pair p), so they are
+// numbered from the most expensive pair level down (unit = level * BH + bh, pair = pairs-1-level)
+// and dealt to the CTAs in snake order (round r gives CTA c the unit r*G + c for even r and
+// r*G + G-1-c for odd r), a static form of longest-processing-time-first scheduling.
 struct WorkUnit {
   int bh;
-  int pairs[2];
-  int count;
+  int pair;
 };
+
+// The unit CTA blockIdx.x processes in its round r, or -1 once it has none left.
+__device__ __forceinline__ int unit_for_round(const PrefillParams &p, int r) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const int u = r * G + ((p.causal && (r & 1)) ? G - 1 - c : c);
+  return u < p.num_units ? u : -1;
+}
 
 __device__ __forceinline__ WorkUnit decode_unit(const PrefillParams &p, int u) {
   WorkUnit w;
   if (p.causal) {
-    const int half = (p.num_pairs + 1) / 2;
-    w.bh = u / half;
-    const int s = u % half;
-    const int partner = p.num_pairs - 1 - s;
-    w.pairs[0] = partner;  // the heavier pair first
-    w.pairs[1] = s;
-    w.count = (partner == s) ? 1 : 2;
+    w.bh = u % p.BH;
+    w.pair = p.num_pairs - 1 - u / p.BH;
   } else {
     w.bh = u / p.num_pairs;
-    w.pairs[0] = u % p.num_pairs;
-    w.pairs[1] = -1;
-    w.count = 1;
+    w.pair = u % p.num_pairs;
   }
   return w;
 }
@@ -119,6 +132,99 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   }
 }
 
+#ifndef FA_PACKED_F32X2
+#define FA_PACKED_F32X2 1
+#endif
+#ifndef FA_P_CHUNKS
+#define FA_P_CHUNKS 0
+#endif
+
+// One row of a score block -> P: p = 2^(s * scale*log2e - m_ref) for the 128 scores of this
+// thread's row (MUFU ex2, or the FMA-pipe polynomial for every kPolyEvery-th pair).  P is written
+// to TMEM as bf16 pairs (2 per 32-bit column), in 16-column chunks as each is ready
+// (FA_P_CHUNKS) or in two 32-column stores at the end.  Returns the sum of the fp32 p (for the LSE)
+// and the sum of the bf16-rounded p that P V actually uses (the normaliser of O, so that O is an
+// exact convex combination of V rows even when one key dominates).  kTrackMax also returns the
+// row's maximum score.
+template <bool kTrackMax>
+__device__ __forceinline__ void exp_row(float (&s)[kBN], float sl2, float mneg, uint32_t tP,
+                                        float &sum_exact, float &sum_rounded, float &smax) {
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#if FA_PACKED_F32X2
+  const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(mneg, mneg);
+  uint64_t le2 = 0, lr2 = 0;
+#else
+  float le0 = 0.f, le1 = 0.f, lr0 = 0.f, lr1 = 0.f;
+#endif
+#if !FA_P_CHUNKS
+  uint32_t pall[kBN / 2];
+#endif
+#pragma unroll
+  for (int g = 0; g < kBN / 32; ++g) {
+#if FA_P_CHUNKS
+    uint32_t pk[16];
+#else
+    uint32_t *pk = pall + g * 16;
+#endif
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int e = g * 32 + 2 * c;
+      if (kTrackMax) {
+        if (c & 1) mx1 = fmax3(mx1, s[e], s[e + 1]);
+        else mx0 = fmax3(mx0, s[e], s[e + 1]);
+      }
+      const bool poly = kPolyEvery > 0 && (g * 16 + c) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1;
+      float p0, p1;
+#if FA_PACKED_F32X2
+      const uint64_t x2 = f2_fma(f2_pack(s[e], s[e + 1]), c2, m2);
+      uint64_t p2;
+      if (poly) {
+        p2 = exp2_poly_x2(x2);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p2 = f2_pack(ex2(x0), ex2(x1));
+      }
+      le2 = f2_add(le2, p2);
+      f2_unpack(p2, p0, p1);
+      pk[c] = pack_bf16x2(p0, p1);
+      lr2 = f2_add(lr2, f2_pack(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
+#else
+      const float x0 = fmaf(s[e], sl2, mneg), x1 = fmaf(s[e + 1], sl2, mneg);
+      if (poly) {
+        f2_unpack(exp2_poly_x2(f2_pack(x0, x1)), p0, p1);
+      } else {
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
+      le0 += p0;
+      le1 += p1;
+      pk[c] = pack_bf16x2(p0, p1);
+      lr0 += __uint_as_float(pk[c] << 16);
+      lr1 += __uint_as_float(pk[c] & 0xffff0000u);
+#endif
+    }
+#if FA_P_CHUNKS
+    tmem_st16(tP + g * 16, pk);
+#endif
+  }
+#if !FA_P_CHUNKS
+  tmem_st32(tP, pall);
+  tmem_st32(tP + 32, pall + 32);
+#endif
+#if FA_PACKED_F32X2
+  float a, b;
+  f2_unpack(le2, a, b);
+  sum_exact = a + b;
+  f2_unpack(lr2, a, b);
+  sum_rounded = a + b;
+#else
+  sum_exact = le0 + le1;
+  sum_rounded = lr0 + lr1;
+#endif
+  smax = fmaxf(mx0, mx1);
+}
+
 template <int HD>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -154,7 +260,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_ready[i], kBM);
+      mbar_init(&p_ready[i], kBM / 32);
       mbar_init(&o_done[i], 1);
     }
     mbar_init(drain, 1);
@@ -175,7 +281,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int nkb = (p.N + kBN - 1) / kBN;
-
+  if (warp >= 8) {
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -185,10 +291,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bool issued[C::kStages];
       for (int s = 0; s < C::kStages; ++s) issued[s] = false;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_super; u += gridDim.x) {
+      for (int r = 0; ok; ++r) {
+        const int u = unit_for_round(p, r);
+        if (u < 0) break;
         const WorkUnit w = decode_unit(p, u);
-        for (int t = 0; ok && t < w.count; ++t) {
-          const int pr = w.pairs[t];
+        {
+          const int pr = w.pair;
           const int n0 = tile_blocks(p, pr, 0), n1 = tile_blocks(p, pr, 1);
           const int nmax = n0 > n1 ? n0 : n1;
           if (!mbar_wait(q_empty, q_ph ^ 1, abort_flag)) { ok = false; break; }
@@ -231,10 +339,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const uint32_t sQ0 = smem_u32(sQ), sQ1 = smem_u32(sQ + C::kTileBytes);
       const uint32_t sKV0 = smem_u32(sKV);
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_super; u += gridDim.x) {
+      for (int r = 0; ok; ++r) {
+        const int u = unit_for_round(p, r);
+        if (u < 0) break;
         const WorkUnit w = decode_unit(p, u);
-        for (int t = 0; ok && t < w.count; ++t) {
-          const int pr = w.pairs[t];
+        {
+          const int pr = w.pair;
           const int n[2] = {tile_blocks(p, pr, 0), tile_blocks(p, pr, 1)};
           const int nmax = n[0] > n[1] ? n[0] : n[1];
           if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
@@ -292,7 +402,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       volatile int never = 0;
       mbar_wait(drain, 0, &never);
     }
-  } else if (warp < 8) {
+  }
+  } else {
     // ------------------------------------------------------------------ softmax / epilogue
     const int wg = warp / 4;                       // which tile of the pair
     const int row = threadIdx.x % 128;             // TMEM lane == query row within the tile
@@ -302,14 +413,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const float sl2 = p.scale_log2;
     uint32_t s_ph = 0, o_ph = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.num_super; u += gridDim.x) {
+    for (int r = 0; ok; ++r) {
+      const int u = unit_for_round(p, r);
+      if (u < 0) break;
       const WorkUnit w = decode_unit(p, u);
-      for (int t = 0; ok && t < w.count; ++t) {
-        const int pr = w.pairs[t];
+      {
+        const int pr = w.pair;
         const int n = tile_blocks(p, pr, wg);
         if (n == 0) continue;
         const int qrow = pr * 2 * kBM + wg * kBM + row;
-        float m_ref = -INFINITY, l = 0.f;
+        float m_ref = -INFINITY, l = 0.f, lr = 0.f;
         for (int j = 0; j < n; ++j) {
           // the decision to go on must be warp-uniform: tcgen05.ld/st below are warp-collective
           if (!__all_sync(0xffffffffu, mbar_wait(&s_full[wg], s_ph, abort_flag))) { ok = false; break; }
@@ -328,36 +441,47 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int c = 0; c < kBN; ++c)
               if (c >= lim) s[c] = -INFINITY;
           }
-          float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+          // Lazy rescale: the reference max m_ref (log2 units) moves only when a block's max
+          // exceeds it by more than 2^8.  After the first block the exponentials are computed
+          // optimistically against the current m_ref while the block max is found in the same
+          // pass; only if some row of the warp moved its reference (rare) is the pass redone.
+          bool need;
+          float alpha, le, lrb, smax;
+          if (j == 0 || !FA_OPTIMISTIC_EXP) {
+            float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
+            float mx2 = fmax3(s[6], s[7], s[8]), mx3 = fmax3(s[9], s[10], s[11]);
 #pragma unroll
-          for (int c = 4; c < kBN; c += 4) {
-            mx0 = fmaxf(mx0, s[c]);
-            mx1 = fmaxf(mx1, s[c + 1]);
-            mx2 = fmaxf(mx2, s[c + 2]);
-            mx3 = fmaxf(mx3, s[c + 3]);
+            for (int c = 12; c < kBN - 8; c += 8) {
+              mx0 = fmax3(mx0, s[c], s[c + 1]);
+              mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+              mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+              mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+            }
+            mx0 = fmax3(mx0, s[kBN - 4], s[kBN - 3]);
+            mx1 = fmax3(mx1, s[kBN - 2], s[kBN - 1]);
+            const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            need = m_blk > m_ref + kRescaleLog2;  // always true on the first block (m_ref = -inf)
+            alpha = 1.f;
+            if (need) {
+              alpha = ex2(m_ref - m_blk);  // 2^-inf = 0 on the first block
+              m_ref = m_blk;
+            }
+            exp_row<false>(s, sl2, (m_ref == -INFINITY) ? 0.f : -m_ref, tS, le, lrb, smax);
+          } else {
+            exp_row<true>(s, sl2, -m_ref, tS, le, lrb, smax);
+            const float m_blk = smax * sl2;
+            need = m_blk > m_ref + kRescaleLog2;
+            alpha = 1.f;
+            if (__any_sync(0xffffffffu, need)) {
+              if (need) {
+                alpha = ex2(m_ref - m_blk);
+                m_ref = m_blk;
+              }
+              exp_row<false>(s, sl2, -m_ref, tS, le, lrb, smax);
+            }
           }
-          const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-          // lazy rescale: move the reference max only when the block max exceeds it by > 2^8
-          const bool need = m_blk > m_ref + kRescaleLog2;
-          const float alpha = need ? ex2(m_ref - m_blk) : 1.f;  // 2^-inf = 0 on the first block
-          if (need) {
-            m_ref = m_blk;
-            l *= alpha;
-          }
-          const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
-          float rs0 = 0.f, rs1 = 0.f;
-          uint32_t pk[kBN / 2];
-#pragma unroll
-          for (int c = 0; c < kBN / 2; ++c) {
-            const float p0 = ex2(fmaf(s[2 * c], sl2, mneg));
-            const float p1 = ex2(fmaf(s[2 * c + 1], sl2, mneg));
-            rs0 += p0;
-            rs1 += p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          tmem_st32(tS + 0, pk);
-          tmem_st32(tS + 32, pk + 32);
-          l += rs0 + rs1;
+          l = l * alpha + le;
+          lr = lr * alpha + lrb;
           if (j > 0 && __any_sync(0xffffffffu, need)) {
             // O_i holds the sum through block j-1 (S_ij's commit covers that MMA): rescale it in
             // place before P_ij V_j is accumulated on top.  Rows that keep their max use alpha 1.
@@ -373,14 +497,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&p_ready[wg]);
+          __syncwarp();
+          if ((threadIdx.x & 31) == 0) mbar_arrive(&p_ready[wg]);  // one arrival per warp
         }
         if (!ok) break;
         // epilogue: O_i / l and LSE once the last P V of this tile has completed
         if (!__all_sync(0xffffffffu, mbar_wait(&o_done[wg], o_ph, abort_flag))) { ok = false; break; }
         o_ph ^= 1;
         tc_fence_after();
-        const float inv = 1.f / l;
+        const float inv = 1.f / lr;
         const bool live = qrow < p.N;
         const size_t grow = static_cast<size_t>(w.bh) * p.N + qrow;
 #pragma unroll
@@ -419,7 +544,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   __syncthreads();
   if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    tmem_dealloc(*tmem_slot, C::kTmemCols);  // the address exactly as the allocation wrote it
   }
 }
 
