@@ -159,11 +159,20 @@ def time_launches(fn, steps, warmup, flush, stream):
 
 
 def dist_max(x: float) -> float:
+    """Max over ranks (every rank calls it at the same point; identity without a process group)."""
     if torch.distributed.is_available() and torch.distributed.is_initialized():
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
     return x
+
+
+def aggregate(step_ms_local: float, flops_per_rank_step: float, world: int):
+    """Whole-job throughput: every rank runs the same independent workload (weak scaling), so the
+    job does world * flops per step in the slowest rank's step time.  Returns (TFLOP/s, max ms)."""
+    step_ms = dist_max(step_ms_local)
+    return world * flops_per_rank_step / (step_ms * 1e-3) / 1e12, step_ms
 
 
 def barrier():
@@ -297,9 +306,8 @@ def bench_ours(args, rank, world):
         for ci, c in enumerate(cases):
             kernel_ms[c.causal].append(evs[st][ci][0].elapsed_time(evs[st][ci][1]))
     step_ms = statistics.mean(kernel_ms[False]) + statistics.mean(kernel_ms[True])
-    step_ms_max = dist_max(step_ms)
     flops_step = sum(c.flops for c in cases)
-    value = world * flops_step / (step_ms_max * 1e-3) / 1e12
+    value, step_ms_max = aggregate(step_ms, flops_step, world)
     peak_key = "bf16_tflops"
     achieved = flops_step / (step_ms * 1e-3) / 1e12
     traffic = committed_traffic("prefill", KERNEL_SOURCES)

@@ -27,7 +27,7 @@ FA_OUT_BF16, FA_OUT_F32 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
                     "fa_decode_paged_noalloc", "fa_get_device_status", "fa_status_string",
-                    "fa_last_error_string", "fa_version")
+                    "fa_last_error_string", "fa_version", "fa_selftest_wait_timeout")
 
 _lib = None
 
@@ -212,3 +212,14 @@ def fa_decode_paged_noalloc(q, k_pool, v_pool, block_table, seq_lens, out, lse=N
            float(scale) if scale is not None else 0.0, _stream_handle(stream))
     _check(st, "fa_decode_paged_noalloc")
     return out, lse
+
+
+def selftest_wait_timeout(limit_us: int = 50_000, stream=None) -> int:
+    """Launch the bounded-wait self-test and return the device status it leaves (expect 5,
+    FA_ERR_TIMEOUT); the status word is read and cleared."""
+    lib = load_library()
+    f = lib.fa_selftest_wait_timeout
+    f.argtypes = [ctypes.c_uint, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    _check(f(limit_us, _stream_handle(stream)), "fa_selftest_wait_timeout")
+    return device_status(stream)

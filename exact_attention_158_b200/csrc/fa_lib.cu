@@ -16,6 +16,19 @@
 #include "fa_decode.cuh"
 #include "fa_prefill.cuh"
 
+namespace fa {
+// One thread waits on a barrier that nothing arrives at; the bounded wait must give up.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0, &abort_flag, limit_ns);  // records FA_ERR_TIMEOUT when it gives up
+}
+}  // namespace fa
+
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
@@ -358,6 +371,18 @@ fa_status fa_get_device_status(fa_stream_t stream) {
       return launch_failed(e);
   }
   return static_cast<fa_status>(v);
+}
+
+fa_status fa_selftest_wait_timeout(unsigned limit_us, fa_stream_t stream) {
+  if (limit_us < 1 || limit_us > 2000000u) return FA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  fa::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : launch_failed(e);
 }
 
 const char *fa_status_string(fa_status status) {

@@ -61,8 +61,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false (and raises *abort)
-// when the wait exceeds the limit or another role of the CTA has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// when the wait exceeds `limit_ns` or another role of the CTA has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = FA_WAIT_LIMIT_NS) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -71,7 +72,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > FA_WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
       atomicExch(&g_device_status, 5 /* FA_ERR_TIMEOUT */);
       return false;

@@ -149,6 +149,15 @@ fa_status fa_decode_paged_noalloc(const void *q, const void *k_pool, const void 
  */
 fa_status fa_get_device_status(fa_stream_t stream);
 
+/*
+ * fa_selftest_wait_timeout -- diagnostic: launches one thread that waits on a barrier nothing ever
+ * signals, through the same bounded wait the attention kernels use, with a limit of `limit_us`
+ * microseconds (1 .. 2000000).  The wait gives up, the kernel records FA_ERR_TIMEOUT in the device
+ * status word and returns, and the context stays usable.  Lets a caller (or a test) confirm that
+ * a stalled kernel is reported through fa_get_device_status instead of hanging the GPU.
+ */
+fa_status fa_selftest_wait_timeout(unsigned limit_us, fa_stream_t stream);
+
 /* Static text for a status code. */
 const char *fa_status_string(fa_status status);
 
