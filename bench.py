@@ -231,7 +231,7 @@ def run_prefill_case(fa, case, steps, warmup, flush, stream, out_dtype=torch.bfl
 
 
 def bench_decode(fa, args, dev, flush, stream, pk):
-    case = W.DecodeCase("decode")
+    case = W.DecodeCase("decode", S=args.decode_seqs)
     inp = W.make_decode(case, device=dev)
     o = torch.empty_like(inp["q"])
     lse = torch.empty(inp["q"].shape[:2], dtype=torch.float32, device=dev)
@@ -248,7 +248,7 @@ def bench_decode(fa, args, dev, flush, stream, pk):
     ms = statistics.median(ts)
     nbytes = W.decode_bytes(inp["lens"], case.H, case.d, inp["max_blocks"])
     gbs = nbytes / (ms * 1e-3) / 1e9
-    return {"metric": "paged decode GB/s", "workload": "64 seqs, q len 1, H32 d128, "
+    return {"metric": "paged decode GB/s", "workload": f"{case.S} seqs, q len 1, H32 d128, "
             "context U[512,8192], 16-token pages, permuted block table",
             "ms": round(ms, 4), "value": round(gbs, 1), "unit": "GB/s",
             "algorithmic_bytes": nbytes, "tokens": sum(inp["lens"]),
@@ -413,6 +413,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-seqs", type=int, default=64,
+                    help="sequences in the decode workload (64 is the benchmark; fewer for profiling)")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="prefill: the headline loop alone; decode: the decode loop alone")
     args = ap.parse_args()
