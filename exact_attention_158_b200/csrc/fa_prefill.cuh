@@ -48,6 +48,9 @@ struct PrefillCfg {
   // P lives in TMEM when there is room for it beside S and O (d = 64: S 2x128 + O 2x64 + P 2x64
   // columns = 512), otherwise in shared memory (d = 128: S and O fill all 512 columns).
   static constexpr bool kPInTmem = HD == 64;
+  // MMA issue order: at d = 64 an event-driven loop (issue whatever S or P V is ready) measured
+  // faster; at d = 128 the fixed order S_0,j+1  S_1,j+1  PV_0,j  PV_1,j did.
+  static constexpr bool kEventMma = HD == 64;
   static constexpr int kPBytes = kPInTmem ? 0 : 128 * kBN * 2;  // one 128 x 128 bf16 P tile
   // K/V ring depth: K_{j+1} is loaded one block ahead of V_j, so three stages give every load
   // about one block of slack.
@@ -340,76 +343,173 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t kv_it = 0, q_ph = 0;
-      uint32_t s_cnt[2] = {0, 0};  // S_i computed so far (s_free phases follow it)
-      uint32_t p_cnt[2] = {0, 0};  // P_i consumed so far
-      const uint32_t sQ0 = smem_u32(sQ), sQ1 = smem_u32(sQ + C::kTileBytes);
-      const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
-      bool ok = true;
-      // S_i = Q_i K^T into S_i's TMEM columns, once the softmax has copied out the previous S_i.
-      auto issue_s = [&](int i, uint32_t k_stage) -> bool {
-        if (s_cnt[i] > 0 && !mbar_wait(&s_free[i], (s_cnt[i] - 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        issue_qk<HD>(tmem + (i ? C::kColS1 : C::kColS0), i ? sQ1 : sQ0,
-                     sKV0 + k_stage * C::kTileBytes);
-        umma_commit(&s_full[i]);
-        ++s_cnt[i];
-        return true;
-      };
-      for (int r = 0; ok; ++r) {
-        const int u = unit_for_round(p, r);
-        if (u < 0) break;
-        const WorkUnit w = decode_unit(p, u);
-        const int pr = w.pair;
-        const int n[2] = {tile_blocks(p, pr, 0), tile_blocks(p, pr, 1)};
-        const int nmax = n[0] > n[1] ? n[0] : n[1];
-        if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
-        q_ph ^= 1;
-        {
-          const uint32_t st = kv_it % C::kStages, ph = (kv_it / C::kStages) & 1;
-          if (!mbar_wait(&kv_full[st], ph, abort_flag)) { ok = false; break; }
-          for (int i = 0; ok && i < 2; ++i)
-            if (n[i] > 0 && !issue_s(i, st)) ok = false;
-          if (!ok) break;
-          umma_commit(&kv_empty[st]);  // K_0 is free once both S_i,0 have been computed
-          ++kv_it;
-          if (nmax == 1) umma_commit(q_empty);
+    if constexpr (C::kEventMma) {
+      // Event-driven: each pass polls (without blocking) what each tile can take next -- S_i,j once
+      // K_j has landed and the softmax has copied out S_i,j-1, or O_i += P_i,j V_j once V_j has
+      // landed and P_i,j is written -- and issues whatever is ready, scores first, so that neither
+      // tile's softmax waits behind the other tile's work.  Per unit the loads arrive in the order
+      // K_0, then K_{j+1}, V_j for j = 0, 1, ...: load index of K_j is 2j-1 (K_0: 0), of V_j 2j+2
+      // (2j+1 for the last block, which has no K_{j+1} before it).  A load is only tested once the
+      // earlier load that used its stage has landed (its consumer was issued first), so the parity
+      // test cannot see a stale phase.
+      if (lane == 0) {
+        uint32_t kv_base = 0, q_ph = 0;
+        uint32_t s_cnt[2] = {0, 0};  // S_i computed so far (s_free phases follow it)
+        uint32_t p_cnt[2] = {0, 0};  // P_i consumed so far (p_full phases follow it)
+        const uint32_t sQ0 = smem_u32(sQ), sQ1 = smem_u32(sQ + C::kTileBytes);
+        const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+          const int u = unit_for_round(p, r);
+          if (u < 0) break;
+          const WorkUnit w = decode_unit(p, u);
+          const int pr = w.pair;
+          const int n[2] = {tile_blocks(p, pr, 0), tile_blocks(p, pr, 1)};
+          const int nmax = n[0] > n[1] ? n[0] : n[1];
+          if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
+          q_ph ^= 1;
+          tc_fence_after();
+          int s_next[2] = {0, 0}, pv_next[2] = {0, 0};
+          int s_left = n[0] + n[1], pv_left = n[0] + n[1];
+          auto k_load = [&](int j) { return kv_base + (j == 0 ? 0u : static_cast<uint32_t>(2 * j - 1)); };
+          auto v_load = [&](int j) {
+            return kv_base + static_cast<uint32_t>(j + 1 < nmax ? 2 * j + 2 : 2 * j + 1);
+          };
+          auto landed = [&](uint32_t ld) {
+            return mbar_test(&kv_full[ld % C::kStages], (ld / C::kStages) & 1);
+          };
+          uint64_t t_last = globaltimer_ns();
+          while (pv_left > 0) {
+            bool progressed = false;
+            for (int i = 0; i < 2; ++i) {
+              const int j = s_next[i];
+              if (j >= n[i]) continue;
+              const uint32_t kld = k_load(j);
+              if (!landed(kld)) continue;
+              if (s_cnt[i] > 0 && !mbar_test(&s_free[i], (s_cnt[i] - 1) & 1)) continue;
+              tc_fence_after();
+              issue_qk<HD>(tmem + (i ? C::kColS1 : C::kColS0), i ? sQ1 : sQ0,
+                           sKV0 + (kld % C::kStages) * C::kTileBytes);
+              umma_commit(&s_full[i]);
+              ++s_cnt[i];
+              ++s_next[i];
+              --s_left;
+              progressed = true;
+              // K_j is free once every tile that visits block j has computed its S_i,j
+              const int other = s_next[i ^ 1];
+              if (j >= n[i ^ 1] || other > j) umma_commit(&kv_empty[kld % C::kStages]);
+              if (s_left == 0) umma_commit(q_empty);  // every Q K^T of the unit is issued
+            }
+            for (int i = 0; i < 2; ++i) {
+              const int j = pv_next[i];
+              if (j >= n[i] || j >= s_next[i]) continue;
+              const uint32_t vld = v_load(j);
+              if (!landed(vld)) continue;
+              if (!mbar_test(&p_full[i], p_cnt[i] & 1)) continue;
+              ++p_cnt[i];
+              tc_fence_after();
+              const uint32_t p_addr = C::kPInTmem ? tmem + (i ? C::kColP1 : C::kColP0)
+                                                  : sP0 + i * C::kPBytes;
+              issue_pv<HD>(tmem + (i ? C::kColO1 : C::kColO0), p_addr,
+                           sKV0 + (vld % C::kStages) * C::kTileBytes, j > 0);
+              umma_commit(&pv_done[i]);
+              ++pv_next[i];
+              --pv_left;
+              progressed = true;
+              const int other = pv_next[i ^ 1];
+              if (j >= n[i ^ 1] || other > j) umma_commit(&kv_empty[vld % C::kStages]);
+            }
+            if (progressed) {
+              t_last = globaltimer_ns();
+            } else {
+              if (*abort_flag) { ok = false; break; }
+              if (globaltimer_ns() - t_last > FA_WAIT_LIMIT_NS) {
+                *abort_flag = 1;
+                atomicExch(&g_device_status, 5 /* FA_ERR_TIMEOUT */);
+                ok = false;
+                break;
+              }
+            }
+          }
+          kv_base += 2 * nmax;
         }
-        for (int j = 0; ok && j < nmax; ++j) {
-          if (j + 1 < nmax) {
-            // the next scores first: they only need K_{j+1} and the softmax's copy of S_i,j
+        // every MMA issued by this thread completes before TMEM is released
+        umma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never);
+      }
+    } else {
+      if (lane == 0) {
+        uint32_t kv_it = 0, q_ph = 0;
+        uint32_t s_cnt[2] = {0, 0};  // S_i computed so far (s_free phases follow it)
+        uint32_t p_cnt[2] = {0, 0};  // P_i consumed so far
+        const uint32_t sQ0 = smem_u32(sQ), sQ1 = smem_u32(sQ + C::kTileBytes);
+        const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
+        bool ok = true;
+        // S_i = Q_i K^T into S_i's TMEM columns, once the softmax has copied out the previous S_i.
+        auto issue_s = [&](int i, uint32_t k_stage) -> bool {
+          if (s_cnt[i] > 0 && !mbar_wait(&s_free[i], (s_cnt[i] - 1) & 1, abort_flag)) return false;
+          tc_fence_after();
+          issue_qk<HD>(tmem + (i ? C::kColS1 : C::kColS0), i ? sQ1 : sQ0,
+                       sKV0 + k_stage * C::kTileBytes);
+          umma_commit(&s_full[i]);
+          ++s_cnt[i];
+          return true;
+        };
+        for (int r = 0; ok; ++r) {
+          const int u = unit_for_round(p, r);
+          if (u < 0) break;
+          const WorkUnit w = decode_unit(p, u);
+          const int pr = w.pair;
+          const int n[2] = {tile_blocks(p, pr, 0), tile_blocks(p, pr, 1)};
+          const int nmax = n[0] > n[1] ? n[0] : n[1];
+          if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
+          q_ph ^= 1;
+          {
             const uint32_t st = kv_it % C::kStages, ph = (kv_it / C::kStages) & 1;
             if (!mbar_wait(&kv_full[st], ph, abort_flag)) { ok = false; break; }
             for (int i = 0; ok && i < 2; ++i)
-              if (j + 1 < n[i] && !issue_s(i, st)) ok = false;
+              if (n[i] > 0 && !issue_s(i, st)) ok = false;
             if (!ok) break;
-            umma_commit(&kv_empty[st]);
+            umma_commit(&kv_empty[st]);  // K_0 is free once both S_i,0 have been computed
             ++kv_it;
-            if (j + 2 == nmax) umma_commit(q_empty);  // that was the last Q K^T of the unit
+            if (nmax == 1) umma_commit(q_empty);
           }
-          const uint32_t vst = kv_it % C::kStages, vph = (kv_it / C::kStages) & 1;
-          if (!mbar_wait(&kv_full[vst], vph, abort_flag)) { ok = false; break; }
-          for (int i = 0; ok && i < 2; ++i) {
-            if (j >= n[i]) continue;
-            if (!mbar_wait(&p_full[i], p_cnt[i] & 1, abort_flag)) { ok = false; break; }
-            ++p_cnt[i];
-            tc_fence_after();
-            const uint32_t p_addr = C::kPInTmem ? tmem + (i ? C::kColP1 : C::kColP0)
-                                                : sP0 + i * C::kPBytes;
-            issue_pv<HD>(tmem + (i ? C::kColO1 : C::kColO0), p_addr, sKV0 + vst * C::kTileBytes,
-                         j > 0);
-            umma_commit(&pv_done[i]);
+          for (int j = 0; ok && j < nmax; ++j) {
+            if (j + 1 < nmax) {
+              // the next scores first: they only need K_{j+1} and the softmax's copy of S_i,j
+              const uint32_t st = kv_it % C::kStages, ph = (kv_it / C::kStages) & 1;
+              if (!mbar_wait(&kv_full[st], ph, abort_flag)) { ok = false; break; }
+              for (int i = 0; ok && i < 2; ++i)
+                if (j + 1 < n[i] && !issue_s(i, st)) ok = false;
+              if (!ok) break;
+              umma_commit(&kv_empty[st]);
+              ++kv_it;
+              if (j + 2 == nmax) umma_commit(q_empty);  // that was the last Q K^T of the unit
+            }
+            const uint32_t vst = kv_it % C::kStages, vph = (kv_it / C::kStages) & 1;
+            if (!mbar_wait(&kv_full[vst], vph, abort_flag)) { ok = false; break; }
+            for (int i = 0; ok && i < 2; ++i) {
+              if (j >= n[i]) continue;
+              if (!mbar_wait(&p_full[i], p_cnt[i] & 1, abort_flag)) { ok = false; break; }
+              ++p_cnt[i];
+              tc_fence_after();
+              const uint32_t p_addr = C::kPInTmem ? tmem + (i ? C::kColP1 : C::kColP0)
+                                                  : sP0 + i * C::kPBytes;
+              issue_pv<HD>(tmem + (i ? C::kColO1 : C::kColO0), p_addr, sKV0 + vst * C::kTileBytes,
+                           j > 0);
+              umma_commit(&pv_done[i]);
+            }
+            if (!ok) break;
+            umma_commit(&kv_empty[vst]);
+            ++kv_it;
           }
-          if (!ok) break;
-          umma_commit(&kv_empty[vst]);
-          ++kv_it;
         }
+        // every MMA issued by this thread completes before TMEM is released
+        umma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never);
       }
-      // every MMA issued by this thread completes before TMEM is released
-      umma_commit(drain);
-      volatile int never = 0;
-      mbar_wait(drain, 0, &never);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax / epilogue
