@@ -28,6 +28,11 @@
  * oracle_decode_paged gathers one sequence's keys and values through its block table (a logical
  * block k of sequence s lives in physical block block_table[s][k]; "LLM study notes", paged
  * attention) and applies the same plain row definition to the gathered rows.
+ *
+ * oracle_prefill_paged does the same for a chunk of Lq queries per sequence: the queries are the
+ * last Lq positions of the sequence's L cached tokens ("Paged vs Flash attention": paging for the
+ * cache, exact attention for the compute), so query t of the chunk sits at position L - Lq + t and,
+ * when causal, sees keys 0 .. L - Lq + t; otherwise all L keys.
  */
 #include <math.h>
 #include <pthread.h>
@@ -319,6 +324,75 @@ int oracle_decode_paged(const uint16_t *q, const uint16_t *k_pool, const uint16_
                      o, lse, units * t / nthreads, units * (t + 1) / nthreads};
         jobs[t] = j;
         pthread_create(&th[t], NULL, dec_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+    free(jobs);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* chunked prefill over a paged cache: Lq queries per sequence, the last Lq of its L tokens     */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *q, *kp, *vp;
+    const int32_t *table, *lens;
+    int max_blocks, H, Lq, d, page, causal;
+    double scale;
+    double *o, *lse;
+    int64_t first, last; /* range of (s, h, t) rows */
+} pf_job;
+
+static void *pf_worker(void *arg)
+{
+    pf_job *jb = (pf_job *)arg;
+    const int H = jb->H, d = jb->d, page = jb->page, Lq = jb->Lq;
+    int64_t maxlen = (int64_t)jb->max_blocks * page;
+    double *s = (double *)malloc(sizeof(double) * (size_t)maxlen);
+    const uint16_t **kr = (const uint16_t **)malloc(sizeof(void *) * (size_t)maxlen);
+    const uint16_t **vr = (const uint16_t **)malloc(sizeof(void *) * (size_t)maxlen);
+    for (int64_t r = jb->first; r < jb->last; ++r) {
+        int64_t t = r % Lq, u = r / Lq, sq = u / H, h = u % H;
+        int64_t L = jb->lens[sq];
+        int64_t n_keys = jb->causal ? L - Lq + t + 1 : L;
+        for (int64_t k = 0; k < n_keys; ++k) {
+            int64_t blk = jb->table[sq * jb->max_blocks + k / page];
+            int64_t off = ((blk * H + h) * page + k % page) * d;
+            kr[k] = jb->kp + off;
+            vr[k] = jb->vp + off;
+        }
+        attend_row(jb->q + r * d, kr, vr, n_keys, d, jb->scale, s, jb->o + r * d, jb->lse + r);
+    }
+    free(s);
+    free(kr);
+    free(vr);
+    return NULL;
+}
+
+/* q [S,H,Lq,d]; pools [num_blocks,H,page,d]; table [S,max_blocks]; lens [S] (each >= Lq);
+ * o [S,H,Lq,d]; lse [S,H,Lq]. */
+int oracle_prefill_paged(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool,
+                         const int32_t *block_table, int max_blocks, const int32_t *seq_lens, int S,
+                         int H, int Lq, int d, int page, int causal, double scale, double *o,
+                         double *lse, int nthreads)
+{
+    if (S < 1 || H < 1 || Lq < 1 || d < 1 || page < 1 || max_blocks < 1 || nthreads < 1)
+        return 1;
+    for (int s = 0; s < S; ++s)
+        if (seq_lens[s] < Lq || seq_lens[s] > (int64_t)max_blocks * page)
+            return 1;
+    int64_t rows = (int64_t)S * H * Lq;
+    if (nthreads > rows)
+        nthreads = (int)rows;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    pf_job *jobs = (pf_job *)malloc(sizeof(pf_job) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) {
+        pf_job j = {q, k_pool, v_pool, block_table, seq_lens, max_blocks, H, Lq, d, page, causal,
+                    scale, o, lse, rows * t / nthreads, rows * (t + 1) / nthreads};
+        jobs[t] = j;
+        pthread_create(&th[t], NULL, pf_worker, &jobs[t]);
     }
     for (int t = 0; t < nthreads; ++t)
         pthread_join(th[t], NULL);

@@ -52,8 +52,10 @@ class OracleLib:
                                           _f64p, _f64p, _f64p]
         lib.oracle_decode_paged.argtypes = [_u16p, _u16p, _u16p, _i32p, _int, _i32p, _int, _int,
                                             _int, _int, _dbl, _f64p, _f64p, _int]
+        lib.oracle_prefill_paged.argtypes = [_u16p, _u16p, _u16p, _i32p, _int, _i32p, _int, _int,
+                                             _int, _int, _int, _int, _dbl, _f64p, _f64p, _int]
         for f in (lib.oracle_attention, lib.oracle_attention_rows, lib.oracle_attention_probs,
-                  lib.oracle_flash_alg1, lib.oracle_decode_paged):
+                  lib.oracle_flash_alg1, lib.oracle_decode_paged, lib.oracle_prefill_paged):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -123,6 +125,25 @@ class OracleLib:
         return o, lse
 
 
+    def prefill_paged(self, q, k_pool, v_pool, block_table, seq_lens, causal: bool, scale: float,
+                      page: int = 16, nthreads: int | None = None):
+        """Chunked prefill over a paged cache.  q [S,H,Lq,d] are the last Lq positions of each
+        sequence's context; pools [P,H,page,d]; block_table int32 [S,max_blocks]; seq_lens int32
+        [S] (each >= Lq).  Returns (o [S,H,Lq,d], lse [S,H,Lq])."""
+        q, k_pool, v_pool = _bits(q), _bits(k_pool), _bits(v_pool)
+        table = np.ascontiguousarray(block_table, dtype=np.int32)
+        lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        S, H, Lq, d = q.shape
+        o = np.empty((S, H, Lq, d), np.float64)
+        lse = np.empty((S, H, Lq), np.float64)
+        rc = self.lib.oracle_prefill_paged(q, k_pool, v_pool, table, table.shape[1], lens, S, H,
+                                           Lq, d, page, int(causal), scale, o, lse,
+                                           nthreads or default_threads())
+        if rc:
+            raise ValueError("oracle_prefill_paged: bad arguments")
+        return o, lse
+
+
 def default_threads() -> int:
     return max(1, len(os.sched_getaffinity(0)))
 
@@ -160,3 +181,7 @@ def flash_alg1(*a, **kw):
 
 def decode_paged(*a, **kw):
     return default().decode_paged(*a, **kw)
+
+
+def prefill_paged(*a, **kw):
+    return default().prefill_paged(*a, **kw)

@@ -262,6 +262,52 @@ def pin_paged_decode(orc):
     close(lse2, lse, 0.0, "relocated pool LSE")
 
 
+def _gather(kp, vp, table, s, h, L, page=16):
+    rows = [(int(table[s, t // page]), t % page) for t in range(L)]
+    return np.stack([kp[b, h, r] for b, r in rows]), np.stack([vp[b, h, r] for b, r in rows])
+
+
+def pin_paged_prefill(orc):
+    """Chunked prefill over a paged cache: query t of the chunk sits at position L - Lq + t; causal
+    rows see keys 0 .. L - Lq + t of the gathered context (softmax/logsumexp from scipy); the
+    last row is the decode step; Lq = L with the whole context is causal attention over it."""
+    case = W.DecodeCase("pinpf", S=3, H=2, d=16, lens=[20, 33, 47])
+    for Lq in (1, 7, 20):
+        inp = W.make_paged_prefill(case, Lq)
+        q = W.bf16_bits(inp["q"])
+        kp, vp = W.bf16_bits(inp["k_pool"]), W.bf16_bits(inp["v_pool"])
+        table, lens = inp["block_table"].numpy(), inp["seq_lens"].numpy()
+        for causal in (True, False):
+            o, lse = orc.prefill_paged(q, kp, vp, table, lens, causal, case.scale)
+            for s, L in enumerate(case.lens):
+                for h in range(case.H):
+                    Kc, Vc = _gather(kp, vp, table, s, h, L)
+                    S_ = case.scale * widen(q[s, h]) @ widen(Kc).T
+                    if causal:
+                        for t in range(Lq):
+                            S_[t, L - Lq + t + 1:] = -np.inf
+                    close(o[s, h], sps.softmax(S_, axis=1) @ widen(Vc), 1e-13,
+                          f"paged prefill O Lq={Lq} causal={causal} s={s} h={h}")
+                    close(lse[s, h], sps.logsumexp(S_, axis=1), 1e-13,
+                          f"paged prefill LSE Lq={Lq} causal={causal} s={s} h={h}")
+            if Lq == 1 and causal:
+                od, ld = orc.decode_paged(q[:, :, 0].copy(), kp, vp, table, lens, case.scale)
+                close(o[:, :, 0], od, 1e-15, "paged prefill Lq=1 vs decode")
+                close(lse[:, :, 0], ld, 1e-15, "paged prefill Lq=1 vs decode LSE")
+    # Lq = L over one sequence: plain causal attention over the gathered rows
+    case1 = W.DecodeCase("pinpf1", S=1, H=2, d=16, lens=[37])
+    inp = W.make_paged_prefill(case1, 37)
+    q = W.bf16_bits(inp["q"])
+    kp, vp = W.bf16_bits(inp["k_pool"]), W.bf16_bits(inp["v_pool"])
+    table, lens = inp["block_table"].numpy(), inp["seq_lens"].numpy()
+    o, lse = orc.prefill_paged(q, kp, vp, table, lens, True, case1.scale)
+    for h in range(2):
+        Kc, Vc = _gather(kp, vp, table, 0, h, 37)
+        oc, lc = orc.attention(q[0, h].copy(), Kc, Vc, True, case1.scale)
+        close(o[0, h], oc, 1e-13, "paged prefill Lq=L vs causal attention")
+        close(lse[0, h], lc, 1e-13, "paged prefill Lq=L vs causal attention LSE")
+
+
 ALL_PINS = [pin_uniform_scores, pin_single_key, pin_dominant_score, pin_two_keys_logistic,
             pin_shift_invariance, pin_rows_sum_to_one, pin_library_softmax, pin_permutation,
-            pin_linear_in_v, pin_tiled_algorithm, pin_paged_decode]
+            pin_linear_in_v, pin_tiled_algorithm, pin_paged_decode, pin_paged_prefill]

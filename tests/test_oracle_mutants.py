@@ -34,6 +34,10 @@ MUTANTS = {
                        "double l_new = l[qi] + a_new * lt;"),
     "tiled_mask_edge": ("vis = last + 1;", "vis = last > 0 ? last : 1;"),
     "probs_no_norm": ("row[j] /= l;", "row[j] /= 1.0;"),
+    "chunk_causal_offset": ("int64_t n_keys = jb->causal ? L - Lq + t + 1 : L;",
+                            "int64_t n_keys = jb->causal ? L - Lq + t : L;"),
+    "chunk_query_row": ("attend_row(jb->q + r * d, kr, vr, n_keys, d, jb->scale, s, jb->o + r * d, jb->lse + r);",
+                        "attend_row(jb->q + (r - t) * d, kr, vr, n_keys, d, jb->scale, s, jb->o + r * d, jb->lse + r);"),
 }
 
 

@@ -255,6 +255,18 @@ def make_decode(case: DecodeCase, device="cpu"):
                 seq_lens=seq_lens.to(device), num_blocks=P, max_blocks=maxb, lens=lens)
 
 
+def make_paged_prefill(case: DecodeCase, Lq: int, device="cpu"):
+    """Chunked prefill over a paged cache: the decode case's pool, table and lengths (each length
+    must be >= Lq), plus q [S,H,Lq,d] for the last Lq positions of every sequence."""
+    inp = make_decode(case, device)
+    if min(inp["lens"]) < Lq:
+        raise ValueError("every context must hold the Lq chunk")
+    inp["q"] = normal_bf16(case.seed, TID_Q, case.S * case.H * Lq * case.d, device).view(
+        case.S, case.H, Lq, case.d)
+    inp["Lq"] = Lq
+    return inp
+
+
 def decode_bytes(lens, H: int, d: int, max_blocks: int) -> int:
     """Algorithmic bytes of one paged decode pass: K and V of every context token (bf16), q and o
     (bf16), the block-table entries actually used (int32) and the lengths (int32)."""
