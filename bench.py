@@ -14,7 +14,8 @@ independent, so there is no collective on the data path).
 Extra keys: `roofline` (prefill kernel vs the measured dense bf16 peak), `cpu_baseline` (the fp64
 oracle on this host's cores, a bounded row sample), `e2e` (the same metric through the Python API
 with Q/K/V copied from pinned host memory and O/LSE copied back inside the timed region), `sweep`
-(the sequence-length grid, d = 128 and d = 64), `decode` (paged decode GB/s vs HBM) and `clocks`.
+(the sequence-length grid, d = 128 and d = 64), `decode` (paged decode GB/s vs HBM),
+`paged_prefill` (chunked prefill through the block table, TFLOP/s) and `clocks`.
 """
 from __future__ import annotations
 
@@ -258,6 +259,32 @@ def bench_decode(fa, args, dev, flush, stream, pk):
             "launches_per_step": 2}
 
 
+def bench_paged_prefill(fa, args, dev, flush, stream, pk):
+    case = W.DecodeCase("paged_prefill", S=16, H=32, d=128, len_lo=2048, len_hi=8192)
+    Lq = 512
+    inp = W.make_paged_prefill(case, Lq, device=dev)
+    o = torch.empty_like(inp["q"])
+    lse = torch.empty(inp["q"].shape[:3], dtype=torch.float32, device=dev)
+    fn = lambda: fa.fa_prefill_paged(inp["q"], inp["k_pool"], inp["v_pool"], inp["block_table"],
+                                     inp["seq_lens"], causal=True, scale=case.scale, out=o,
+                                     lse=lse)
+    torch.cuda.nvtx.range_push("bench_paged_prefill_timed")
+    ts = time_launches(fn, args.sweep_steps, 3, flush, stream)
+    torch.cuda.nvtx.range_pop()
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during the paged prefill bench")
+    ms = statistics.median(ts)
+    flops = W.paged_prefill_flops(inp["lens"], case.H, case.d, Lq, True)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"metric": "chunked prefill over a paged cache, TFLOP/s",
+            "workload": f"{case.S} seqs, chunk {Lq}, H32 d128, context U[2048,8192], "
+            "16-token pages, permuted block table, causal (bottom-right)",
+            "ms": round(ms, 4), "value": round(tf, 1), "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / pk["bf16_tflops"], 4)},
+            "launches_per_step": 1}
+
+
 def bench_ours(args, rank, world):
     import exact_attention_158_b200 as fa
     fa.load_library()
@@ -267,6 +294,9 @@ def bench_ours(args, rank, world):
     pk = peaks()
     if args.only == "decode":
         return {"metric": METRIC, "decode": bench_decode(fa, args, dev, flush, stream, pk)}
+    if args.only == "paged":
+        return {"metric": METRIC,
+                "paged_prefill": bench_paged_prefill(fa, args, dev, flush, stream, pk)}
 
     # ---- headline: prefill config, non-causal + causal per step
     cases = W.prefill_cases()
@@ -382,7 +412,10 @@ def bench_ours(args, rank, world):
     # ---- paged decode (HBM bound)
     dec = None if args.no_decode else bench_decode(fa, args, dev, flush, stream, pk)
 
-    result.update({"e2e": e2e, "sweep": sweep, "decode": dec})
+    # ---- chunked prefill over the paged cache (tensor bound)
+    paged = None if args.no_paged else bench_paged_prefill(fa, args, dev, flush, stream, pk)
+
+    result.update({"e2e": e2e, "sweep": sweep, "decode": dec, "paged_prefill": paged})
     return result
 
 
@@ -415,11 +448,13 @@ def main():
     ap.add_argument("--sweep-steps", type=int, default=20)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-paged", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="sequences in the decode workload (64 is the benchmark; fewer for profiling)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
-                    help="prefill: the headline loop alone; decode: the decode loop alone")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "paged"], default="all",
+                    help="prefill: the headline loop alone; decode / paged: the paged decode or "
+                    "chunked prefill loop alone")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

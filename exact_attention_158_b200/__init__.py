@@ -17,7 +17,8 @@ import torch
 
 from . import build as _build
 
-__all__ = ["fa_fwd", "fa_decode_paged", "fa_decode_paged_noalloc", "fa_decode_workspace_size",
+__all__ = ["fa_fwd", "fa_decode_paged", "fa_decode_paged_noalloc", "fa_prefill_paged",
+           "fa_decode_workspace_size",
            "NOALLOC_SCRATCH_BYTES", "device_status",
            "FaError", "library_path", "load_library", "EXPORTED_SYMBOLS", "STATUS"]
 
@@ -26,7 +27,8 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 FA_OUT_BF16, FA_OUT_F32 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
-                    "fa_decode_paged_noalloc", "fa_get_device_status", "fa_status_string",
+                    "fa_decode_paged_noalloc", "fa_prefill_paged", "fa_get_device_status",
+                    "fa_status_string",
                     "fa_last_error_string", "fa_version", "fa_selftest_wait_timeout")
 
 _lib = None
@@ -65,6 +67,9 @@ def load_library():
     lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, i32, vp, i32, i32, i32, f32,
                                     vp, sz, vp]
     lib.fa_decode_paged.restype = i32
+    lib.fa_prefill_paged.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, i32, vp, i32, i32, i32, i32,
+                                     i32, f32, vp]
+    lib.fa_prefill_paged.restype = i32
     lib.fa_get_device_status.argtypes = [vp]
     lib.fa_get_device_status.restype = i32
     lib.fa_status_string.argtypes = [i32]
@@ -176,6 +181,40 @@ def fa_decode_paged(q, k_pool, v_pool, block_table, seq_lens, scale: float | Non
                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                  _stream_handle(stream))
     _check(st, "fa_decode_paged")
+    return out, lse
+
+
+def fa_prefill_paged(q, k_pool, v_pool, block_table, seq_lens, causal: bool = True,
+                     scale: float | None = None, out_dtype=torch.bfloat16, out=None, lse=None,
+                     return_lse: bool = True, stream=None):
+    """Chunked prefill over a paged KV cache: q bf16 [S, H, Lq, d] holds the last Lq positions of
+    each sequence (their keys/values already in the cache); k_pool, v_pool bf16
+    [num_blocks, H, 16, d]; block_table int32 [S, max_blocks]; seq_lens int32 [S] (each >= Lq).
+    Returns (o [S, H, Lq, d], lse fp32 [S, H, Lq] or None)."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _require(t, n)
+    _require(block_table, "block_table", torch.int32)
+    _require(seq_lens, "seq_lens", torch.int32)
+    S, H, Lq, d = q.shape
+    P = k_pool.shape[0]
+    if k_pool.shape != (P, H, 16, d) or v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool / v_pool must be [num_blocks, H, 16, d]")
+    if block_table.dim() != 2 or block_table.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_table must be [S, max_blocks] and seq_lens [S]")
+    code = _out_code(out_dtype)
+    if out is None:
+        out = torch.empty((S, H, Lq, d), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((S, H, Lq), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib.fa_prefill_paged(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                  block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(),
+                                  P, out.data_ptr(), code,
+                                  lse.data_ptr() if lse is not None else None, S, H, Lq, d,
+                                  int(causal), float(scale) if scale is not None else 0.0,
+                                  _stream_handle(stream))
+    _check(st, "fa_prefill_paged")
     return out, lse
 
 

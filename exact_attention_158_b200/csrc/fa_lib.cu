@@ -45,7 +45,7 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int num_sms = 0;
-  bool prefill_attr[2] = {false, false};
+  bool prefill_attr[4] = {false, false, false, false};  // (d = 64, 128) x (contiguous, paged)
 };
 
 std::mutex g_mutex;
@@ -118,32 +118,34 @@ bool resolve_scale(float scale, int d, float *out) {
   return true;
 }
 
-template <int HD>
-fa_status launch_prefill(DeviceInfo &dev, const void *q, const void *k, const void *v, void *o,
-                         int o_f32, float *lse, int BH, int N, int causal, float scale,
-                         cudaStream_t stream) {
+// The pools [num_blocks, H, 16, d] as a 4-D tensor (d, 16, H, num_blocks) read in 64 x 16 x 1 x 1
+// boxes: one 16-token page of one head per load.
+bool encode_pool(CUtensorMap *map, const void *base, int d, int H, int num_blocks) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), 16, static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(num_blocks)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(16) * d * 2,
+                           static_cast<cuuint64_t>(H) * 16 * d * 2};
+  cuuint32_t box[4] = {64, 16, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int HD, bool kPaged>
+fa_status launch_prefill(DeviceInfo &dev, const CUtensorMap &tq, const CUtensorMap &tk,
+                         const CUtensorMap &tv, fa::PrefillParams p, cudaStream_t stream) {
   using C = fa::PrefillCfg<HD>;
-  CUtensorMap tq, tk, tv;
-  if (!encode_bhnd(&tq, q, HD, N, BH) || !encode_bhnd(&tk, k, HD, N, BH) ||
-      !encode_bhnd(&tv, v, HD, N, BH)) {
-    t_last_error = "cuTensorMapEncodeTiled failed";
-    return FA_ERR_LAUNCH;
-  }
-  fa::PrefillParams p;
-  p.o = o;
-  p.lse = lse;
-  p.o_f32 = o_f32;
-  p.BH = BH;
-  p.N = N;
-  p.causal = causal;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.num_pairs = (N + 2 * fa::kBM - 1) / (2 * fa::kBM);
-  p.num_units = BH * p.num_pairs;
-  const int slot = HD == 128 ? 1 : 0;
+  p.num_pairs = (p.N + 2 * fa::kBM - 1) / (2 * fa::kBM);
+  p.num_units = p.BH * p.num_pairs;
+  const int slot = (HD == 128 ? 1 : 0) + (kPaged ? 2 : 0);
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!dev.prefill_attr[slot]) {
-      cudaError_t e = cudaFuncSetAttribute(fa::fa_prefill_kernel<HD>,
+      cudaError_t e = cudaFuncSetAttribute(fa::fa_prefill_kernel<HD, kPaged>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(C::kSmemBytes));
       if (e != cudaSuccess) return launch_failed(e);
@@ -151,9 +153,31 @@ fa_status launch_prefill(DeviceInfo &dev, const void *q, const void *k, const vo
     }
   }
   const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
-  fa::fa_prefill_kernel<HD><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  fa::fa_prefill_kernel<HD, kPaged><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk,
+                                                                                         tv, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : launch_failed(e);
+}
+
+template <int HD>
+fa_status launch_prefill_dense(DeviceInfo &dev, const void *q, const void *k, const void *v,
+                               void *o, int o_f32, float *lse, int BH, int N, int causal,
+                               float scale, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!encode_bhnd(&tq, q, HD, N, BH) || !encode_bhnd(&tk, k, HD, N, BH) ||
+      !encode_bhnd(&tv, v, HD, N, BH)) {
+    t_last_error = "cuTensorMapEncodeTiled failed";
+    return FA_ERR_LAUNCH;
+  }
+  fa::PrefillParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.o_f32 = o_f32;
+  p.BH = BH;
+  p.N = N;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  return launch_prefill<HD, false>(dev, tq, tk, tv, p, stream);
 }
 
 int decode_splits(int max_blocks) {
@@ -193,8 +217,8 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, fa_out_dt
   if (st != FA_OK) return st;
   const int o_f32 = o_dtype == FA_OUT_F32;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 128) return launch_prefill<128>(*dev, q, k, v, o, o_f32, lse, BH, N, causal, sc, s);
-  return launch_prefill<64>(*dev, q, k, v, o, o_f32, lse, BH, N, causal, sc, s);
+  if (d == 128) return launch_prefill_dense<128>(*dev, q, k, v, o, o_f32, lse, BH, N, causal, sc, s);
+  return launch_prefill_dense<64>(*dev, q, k, v, o, o_f32, lse, BH, N, causal, sc, s);
 }
 
 size_t fa_decode_workspace_size(int num_seqs, int H, int d, int max_blocks_per_seq) {
@@ -357,6 +381,63 @@ fa_status fa_decode_paged_noalloc(const void *q, const void *k_pool, const void 
   }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : launch_failed(e);
+}
+
+fa_status fa_prefill_paged(const void *q, const void *k_pool, const void *v_pool,
+                           const int32_t *block_table, int max_blocks_per_seq,
+                           const int32_t *seq_lens, int num_blocks, void *o, fa_out_dtype o_dtype,
+                           float *lse, int S, int H, int Lq, int d, int causal, float scale,
+                           fa_stream_t stream) {
+  if (!q || !k_pool || !v_pool || !block_table || !seq_lens || !o) return FA_ERR_INVALID_ARG;
+  if (S < 1 || H < 1 || Lq < 1 || max_blocks_per_seq < 1 || num_blocks < 1) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(S) * H * Lq > INT_MAX) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_blocks_per_seq) * fa::kPage > INT_MAX) return FA_ERR_INVALID_ARG;
+  if (Lq > max_blocks_per_seq * fa::kPage) return FA_ERR_INVALID_ARG;
+  float sc;
+  if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o))
+    return FA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  const size_t rows = static_cast<size_t>(S) * H * Lq;
+  const size_t q_bytes = rows * d * 2, o_bytes = rows * d * (o_dtype == FA_OUT_F32 ? 4 : 2);
+  const size_t pool_bytes = static_cast<size_t>(num_blocks) * H * fa::kPage * d * 2;
+  if (overlaps(o, o_bytes, q, q_bytes) || overlaps(o, o_bytes, k_pool, pool_bytes) ||
+      overlaps(o, o_bytes, v_pool, pool_bytes))
+    return FA_ERR_INVALID_ARG;
+  if (lse && (overlaps(lse, rows * 4, o, o_bytes) || overlaps(lse, rows * 4, q, q_bytes)))
+    return FA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  const int BH = S * H;
+  if (!encode_bhnd(&tq, q, d, Lq, BH) || !encode_pool(&tk, k_pool, d, H, num_blocks) ||
+      !encode_pool(&tv, v_pool, d, H, num_blocks)) {
+    t_last_error = "cuTensorMapEncodeTiled failed";
+    return FA_ERR_LAUNCH;
+  }
+  fa::PrefillParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.o_f32 = o_dtype == FA_OUT_F32;
+  p.BH = BH;
+  p.N = Lq;
+  p.causal = causal;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.H = H;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128) return launch_prefill<128, true>(*dev, tq, tk, tv, p, s);
+  return launch_prefill<64, true>(*dev, tq, tk, tv, p, s);
 }
 
 fa_status fa_get_device_status(fa_stream_t stream) {

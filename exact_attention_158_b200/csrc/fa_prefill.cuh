@@ -71,11 +71,34 @@ struct PrefillParams {
   void *o;
   float *lse;
   int o_f32;
-  int BH, N, causal;
-  float scale_log2;  // scale * log2(e)
-  int num_pairs;     // ceil(N / 256)
-  int num_units;     // BH * num_pairs query-tile pairs, scheduled over the persistent CTAs
+  int BH, N, causal;  // N: query rows per (b, h); also the key count unless paged
+  float scale_log2;   // scale * log2(e)
+  int num_pairs;      // ceil(N / 256)
+  int num_units;      // BH * num_pairs query-tile pairs, scheduled over the persistent CTAs
+  // paged mode (chunked prefill over a paged KV cache): the N queries of (s, h) are the last N of
+  // the sequence's L = seq_lens[s] cached tokens, whose 16-token blocks are listed in block_table
+  const int32_t *seq_lens;
+  const int32_t *block_table;
+  int max_blocks, num_blocks, H;
 };
+
+// Key count of unit (b, h) and the position of its first query among the keys.
+struct KvSpan {
+  int L;      // keys
+  int q_off;  // query row r sits at key position q_off + r
+};
+
+template <bool kPaged>
+__device__ __forceinline__ KvSpan kv_span(const PrefillParams &p, int bh) {
+  if constexpr (kPaged) {
+    int L = p.seq_lens[bh / p.H];
+    const int hi = p.max_blocks * 16;
+    L = L < p.N ? p.N : (L > hi ? hi : L);  // out-of-contract lengths are clamped, not trusted
+    return {L, L - p.N};
+  } else {
+    return {p.N, 0};
+  }
+}
 
 // Work units are query-tile pairs (two 128-row tiles of one (b, h) that share every K/V block).
 // Non-causal units all cost the same; they are numbered head-major (unit = bh * pairs + pair) so
@@ -90,15 +113,19 @@ struct WorkUnit {
 };
 
 // The unit CTA blockIdx.x processes in its round r, or -1 once it has none left.
+// (Paged units are numbered head-major like non-causal ones: their costs depend on the device-side
+// sequence lengths, which the host does not see.)
+template <bool kPaged = false>
 __device__ __forceinline__ int unit_for_round(const PrefillParams &p, int r) {
   const int G = gridDim.x, c = blockIdx.x;
-  const int u = r * G + ((p.causal && (r & 1)) ? G - 1 - c : c);
+  const int u = r * G + ((!kPaged && p.causal && (r & 1)) ? G - 1 - c : c);
   return u < p.num_units ? u : -1;
 }
 
+template <bool kPaged = false>
 __device__ __forceinline__ WorkUnit decode_unit(const PrefillParams &p, int u) {
   WorkUnit w;
-  if (p.causal) {
+  if (!kPaged && p.causal) {
     w.bh = u % p.BH;
     w.pair = p.num_pairs - 1 - u / p.BH;
   } else {
@@ -108,12 +135,14 @@ __device__ __forceinline__ WorkUnit decode_unit(const PrefillParams &p, int u) {
   return w;
 }
 
-// Key blocks visited by query tile i (0/1) of pair `pr`: 0 if the tile starts past N.
-__device__ __forceinline__ int tile_blocks(const PrefillParams &p, int pr, int i) {
+// Key blocks visited by query tile i (0/1) of pair `pr`: 0 if the tile starts past the last query;
+// causal tiles stop at the block holding the key of their last row.
+__device__ __forceinline__ int tile_blocks(const PrefillParams &p, const KvSpan &kv, int pr, int i) {
   const int q0 = pr * 2 * kBM + i * kBM;
   if (q0 >= p.N) return 0;
-  const int nkb = (p.N + kBN - 1) / kBN;
-  return p.causal ? (q0 / kBN + 1) : nkb;
+  if (!p.causal) return (kv.L + kBN - 1) / kBN;
+  const int last_key = kv.q_off + min(q0 + kBM, p.N) - 1;
+  return last_key / kBN + 1;
 }
 
 // S (TMEM) = Q (smem, K-major) K^T (smem, K-major), K = HD in steps of 16.
@@ -227,7 +256,9 @@ __device__ __forceinline__ void store_p_row(uint8_t *p_tile, int row, const uint
   }
 }
 
-template <int HD>
+// kPaged: keys and values come from a paged cache (tm_k / tm_v are 4-D maps over the pools
+// [num_blocks, H, 16, d]; a 128-key tile is gathered as eight 16-row pages through the block table).
+template <int HD, bool kPaged>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -285,7 +316,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nkb = (p.N + kBN - 1) / kBN;
 
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
@@ -298,24 +328,53 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bool issued[C::kStages];
       for (int s = 0; s < C::kStages; ++s) issued[s] = false;
       bool ok = true;
+      int kv_len = 0;  // key count of the current unit (paged mode)
       auto load_kv = [&](const CUtensorMap *map, int row, int bh) -> bool {
         const uint32_t st = kv_it % C::kStages, ph = (kv_it / C::kStages) & 1;
         if (!mbar_wait(&kv_empty[st], ph ^ 1, abort_flag)) return false;
         mbar_arrive_expect_tx(&kv_full[st], C::kTileBytes);
-        for (int ch = 0; ch < C::kChunks; ++ch)
-          tma_load_3d(sKV + st * C::kTileBytes + ch * C::kChunkBytes, map, &kv_full[st], ch * 64,
-                      row, bh);
+        if constexpr (kPaged) {
+          // keys row .. row+127 of sequence s live in eight 16-token pages; pages past the
+          // sequence's end (masked by the softmax) read as zeros through an out-of-range block
+          const int sq = bh / p.H, h = bh % p.H;
+          const int npages = (kv_len + 15) / 16;
+          int blk[kBN / 16];
+#pragma unroll
+          for (int r = 0; r < kBN / 16; ++r) {
+            const int page = row / 16 + r;
+            int b = page < npages ? p.block_table[static_cast<size_t>(sq) * p.max_blocks + page]
+                                  : p.num_blocks;
+            if (page < npages && (b < 0 || b >= p.num_blocks)) {
+              atomicExch(&g_device_status, 1 /* FA_ERR_INVALID_ARG: bad block-table entry */);
+              b = p.num_blocks;
+            }
+            blk[r] = b;
+          }
+#pragma unroll
+          for (int r = 0; r < kBN / 16; ++r)
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              tma_load_4d(sKV + st * C::kTileBytes + ch * C::kChunkBytes + r * 16 * 128, map,
+                          &kv_full[st], ch * 64, 0, h, blk[r]);
+        } else {
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            tma_load_3d(sKV + st * C::kTileBytes + ch * C::kChunkBytes, map, &kv_full[st], ch * 64,
+                        row, bh);
+        }
         issued[st] = true;
         last_ph[st] = ph;
         ++kv_it;
         return true;
       };
       for (int r = 0; ok; ++r) {
-        const int u = unit_for_round(p, r);
+        const int u = unit_for_round<kPaged>(p, r);
         if (u < 0) break;
-        const WorkUnit w = decode_unit(p, u);
+        const WorkUnit w = decode_unit<kPaged>(p, u);
         const int pr = w.pair;
-        const int n0 = tile_blocks(p, pr, 0), n1 = tile_blocks(p, pr, 1);
+        const KvSpan kv = kv_span<kPaged>(p, w.bh);
+        kv_len = kv.L;
+        if (kPaged && p.seq_lens[w.bh / p.H] != kv.L)
+          atomicExch(&g_device_status, 1 /* FA_ERR_INVALID_ARG: length outside [Lq, 16*max_blocks] */);
+        const int n0 = tile_blocks(p, kv, pr, 0), n1 = tile_blocks(p, kv, pr, 1);
         const int nmax = n0 > n1 ? n0 : n1;
         if (!mbar_wait(q_empty, q_ph ^ 1, abort_flag)) { ok = false; break; }
         q_ph ^= 1;
@@ -360,11 +419,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
         bool ok = true;
         for (int r = 0; ok; ++r) {
-          const int u = unit_for_round(p, r);
+          const int u = unit_for_round<kPaged>(p, r);
           if (u < 0) break;
-          const WorkUnit w = decode_unit(p, u);
+          const WorkUnit w = decode_unit<kPaged>(p, u);
           const int pr = w.pair;
-          const int n[2] = {tile_blocks(p, pr, 0), tile_blocks(p, pr, 1)};
+          const KvSpan kv = kv_span<kPaged>(p, w.bh);
+          const int n[2] = {tile_blocks(p, kv, pr, 0), tile_blocks(p, kv, pr, 1)};
           const int nmax = n[0] > n[1] ? n[0] : n[1];
           if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
           q_ph ^= 1;
@@ -457,11 +517,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           return true;
         };
         for (int r = 0; ok; ++r) {
-          const int u = unit_for_round(p, r);
+          const int u = unit_for_round<kPaged>(p, r);
           if (u < 0) break;
-          const WorkUnit w = decode_unit(p, u);
+          const WorkUnit w = decode_unit<kPaged>(p, u);
           const int pr = w.pair;
-          const int n[2] = {tile_blocks(p, pr, 0), tile_blocks(p, pr, 1)};
+          const KvSpan kv = kv_span<kPaged>(p, w.bh);
+          const int n[2] = {tile_blocks(p, kv, pr, 0), tile_blocks(p, kv, pr, 1)};
           const int nmax = n[0] > n[1] ? n[0] : n[1];
           if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
           q_ph ^= 1;
@@ -524,11 +585,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t s_ph = 0, pv_ph = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-      const int u = unit_for_round(p, r);
+      const int u = unit_for_round<kPaged>(p, r);
       if (u < 0) break;
-      const WorkUnit w = decode_unit(p, u);
+      const WorkUnit w = decode_unit<kPaged>(p, u);
       const int pr = w.pair;
-      const int n = tile_blocks(p, pr, wg);
+      const KvSpan kv = kv_span<kPaged>(p, w.bh);
+      const int n = tile_blocks(p, kv, pr, wg);
       if (n == 0) continue;
       const int qrow = pr * 2 * kBM + wg * kBM + row;
       float m_ref = -INFINITY, l = 0.f, lr = 0.f;
@@ -547,9 +609,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[wg]);
-        const bool edge = (p.causal && j == n - 1) || (j == nkb - 1 && (p.N % kBN) != 0);
+        // masking only where a block reaches past this tile's first row's last visible key or
+        // past the last key
+        bool edge;
+        if constexpr (kPaged)
+          edge = (p.causal && (j + 1) * kBN - 1 > kv.q_off + pr * 2 * kBM + wg * kBM) ||
+                 ((j + 1) * kBN > kv.L);
+        else  // q_off = 0, L = N: only a causal tile's diagonal block and a ragged last block
+          edge = (p.causal && j == n - 1) || ((j + 1) * kBN > p.N && (p.N % kBN) != 0);
         if (edge) {
-          const int lim = (p.causal ? min(qrow + 1, p.N) : p.N) - j * kBN;  // visible keys
+          const int lim = (p.causal ? min(kv.q_off + qrow + 1, kv.L) : kv.L) - j * kBN;  // visible
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
             if (c >= lim) s[c] = -INFINITY;

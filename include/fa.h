@@ -114,6 +114,36 @@ fa_status fa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
                           size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_prefill_paged -- chunked prefill over a paged KV cache: a chunk of Lq new queries per
+ * sequence attends to that sequence's cached keys and values, read through the block table.
+ *
+ * Paging for the cache, exact tiled attention for the compute ("Paged vs Flash attention", their
+ * combination; "LLM study notes", paged attention: the block table maps a sequence's logical
+ * blocks to physical ones).  The chunk is the last Lq of the sequence's L = seq_lens[s] cached
+ * tokens (its keys and values are already in the cache), so query t sits at position L - Lq + t:
+ * with causal = 1 it sees keys 0 .. L - Lq + t (the mask aligned to the bottom-right of the
+ * L x Lq score block); with causal = 0 it sees all L keys.  Lq = 1 is the decode step.
+ *
+ *   q            bf16 [S, H, Lq, d] contiguous.
+ *   k_pool,
+ *   v_pool       bf16 [num_blocks, H, 16, d] contiguous.
+ *   block_table  int32 [S, max_blocks_per_seq], device; entries for pages < ceil(L/16) must be in
+ *                [0, num_blocks); later entries are never read.  A bad entry is reported through
+ *                fa_get_device_status (FA_ERR_INVALID_ARG) and its page reads as zeros.
+ *   seq_lens     int32 [S], device; each in [Lq, 16 * max_blocks_per_seq] (lengths outside are
+ *                clamped into it and reported the same way).
+ *   o            [S, H, Lq, d], bf16 or fp32 per o_dtype;  lse: fp32 [S, H, Lq] or NULL.
+ *   S, H, Lq     >= 1, Lq <= 16 * max_blocks_per_seq;  d: 64 or 128;  causal 0/1;
+ *   scale        as for fa_fwd.
+ * Returns FA_OK once the kernel is queued.  No workspace.
+ */
+fa_status fa_prefill_paged(const void *q, const void *k_pool, const void *v_pool,
+                           const int32_t *block_table, int max_blocks_per_seq,
+                           const int32_t *seq_lens, int num_blocks, void *o, fa_out_dtype o_dtype,
+                           float *lse, int S, int H, int Lq, int d, int causal, float scale,
+                           fa_stream_t stream);
+
+/*
  * fa_decode_paged_noalloc -- fa_decode_paged without a caller-supplied workspace and without any
  * allocation.  No counterpart in the paper: this is a deployment variant of the same decode step,
  * not part of the method.

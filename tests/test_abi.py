@@ -82,6 +82,24 @@ def test_decode_workspace_and_rejections(lib):
     assert dec(lib, o=8 * A) == 1  # output overlaps the workspace
 
 
+def pp(lib, q=A, table=5 * A, maxb=4, lens=6 * A, P=8, o=7 * A, dt=0, lse=None, S=2, H=2, Lq=16,
+       d=128, causal=1, scale=0.0):
+    return lib.fa_prefill_paged(q, 2 * A, 3 * A, table, maxb, lens, P, o, dt, lse, S, H, Lq, d,
+                                causal, scale, None)
+
+
+def test_prefill_paged_rejections(lib):
+    assert pp(lib, q=None) == 1 and pp(lib, table=None) == 1 and pp(lib, lens=None) == 1
+    assert pp(lib, S=0) == 1 and pp(lib, Lq=0) == 1 and pp(lib, maxb=0) == 1 and pp(lib, P=0) == 1
+    assert pp(lib, Lq=4 * 16 + 1) == 1  # the chunk cannot be longer than a table row maps
+    assert pp(lib, causal=3) == 1 and pp(lib, dt=9) == 1
+    assert pp(lib, d=96) == 2
+    assert pp(lib, scale=float("nan")) == 1
+    assert pp(lib, q=A + 8) == 3 and pp(lib, table=5 * A + 2) == 3 and pp(lib, lens=6 * A + 1) == 3
+    assert pp(lib, o=A + 32) == 1  # output overlaps q
+    assert pp(lib, o=2 * A + 64) == 1  # output overlaps the K pool
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)

@@ -89,3 +89,11 @@ def test_decode_lengths_in_range():
     lens = W.DecodeCase("d").seq_lens()
     assert len(lens) == 64 and min(lens) >= 512 and max(lens) <= 8192
     assert len(set(lens)) > 50
+
+
+def test_paged_prefill_flops_counts_visible_pairs():
+    lens, Lq, H, d = [5, 9, 20], 4, 3, 8
+    for causal in (True, False):
+        pairs = sum(1 for L in lens for t in range(Lq) for key in range(L)
+                    if not causal or key <= L - Lq + t)
+        assert W.paged_prefill_flops(lens, H, d, Lq, causal) == 4 * d * H * pairs

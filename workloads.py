@@ -267,6 +267,15 @@ def make_paged_prefill(case: DecodeCase, Lq: int, device="cpu"):
     return inp
 
 
+def paged_prefill_flops(lens, H: int, d: int, Lq: int, causal: bool) -> int:
+    """Matmul FLOPs of a chunked prefill: 4 d per visible (query, key) pair (Q K^T and P V).  The
+    chunk's query t of a length-L context sees L - Lq + t + 1 keys causally, else all L."""
+    pairs = 0
+    for L in lens:
+        pairs += Lq * (L - Lq) + Lq * (Lq + 1) // 2 if causal else Lq * L
+    return 4 * d * H * pairs
+
+
 def decode_bytes(lens, H: int, d: int, max_blocks: int) -> int:
     """Algorithmic bytes of one paged decode pass: K and V of every context token (bf16), q and o
     (bf16), the block-table entries actually used (int32) and the lengths (int32)."""
