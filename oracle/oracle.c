@@ -33,6 +33,19 @@
  * last Lq positions of the sequence's L cached tokens ("Paged vs Flash attention": paging for the
  * cache, exact attention for the compute), so query t of the chunk sits at position L - Lq + t and,
  * when causal, sees keys 0 .. L - Lq + t; otherwise all L keys.
+ *
+ * oracle_attention_bwd is the backward pass: the gradients of the scalar sum_i dO[i] . O[i] with
+ * respect to Q, K and V for a given dO.  The pages describe the backward only in prose ("Paged vs
+ * Flash attention", training: gradients from the stored intermediate results, block by block;
+ * "LLM study notes" and "Flash Attention" (myungum) section 1: the attention matrix is recomputed
+ * rather than stored), so the oracle is the plain definition, the chain rule through the row
+ * softmax above, evaluated one query row at a time with the row recomputed from Q and K:
+ *
+ *     P[i,j]  = e_j / l                       (the row above; masked keys have no entry)
+ *     dV[j]  += P[i,j] dO[i]
+ *     dP[i,j] = dO[i] . V[j]
+ *     dS[i,j] = P[i,j] (dP[i,j] - sum_k P[i,k] dP[i,k])      (the softmax Jacobian)
+ *     dQ[i]  += scale dS[i,j] K[j],   dK[j] += scale dS[i,j] Q[i]
  */
 #include <math.h>
 #include <pthread.h>
@@ -393,6 +406,113 @@ int oracle_prefill_paged(const uint16_t *q, const uint16_t *k_pool, const uint16
                     scale, o, lse, rows * t / nthreads, rows * (t + 1) / nthreads};
         jobs[t] = j;
         pthread_create(&th[t], NULL, pf_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+    free(jobs);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* backward: dQ, dK, dV of one head at a time (heads are independent)                          */
+/* ------------------------------------------------------------------------------------------ */
+
+/* One head: Q, K, V, dO [N, d]; dq, dk, dv [N, d] (overwritten).  p, dp: scratch of N. */
+static void bwd_head(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *dO,
+                     int64_t N, int d, int causal, double scale, double *dq, double *dk,
+                     double *dv, double *p, double *dp)
+{
+    for (int64_t e = 0; e < N * d; ++e) {
+        dq[e] = 0.0;
+        dk[e] = 0.0;
+        dv[e] = 0.0;
+    }
+    for (int64_t i = 0; i < N; ++i) {
+        const int64_t n_keys = causal ? i + 1 : N; /* the keys row i sees */
+        const uint16_t *qi = Q + i * d, *doi = dO + i * d;
+        /* the probability row, recomputed */
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n_keys; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += widen_bf16(qi[c]) * widen_bf16(K[j * d + c]);
+            p[j] = scale * acc;
+            if (p[j] > m)
+                m = p[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < n_keys; ++j) {
+            p[j] = exp(p[j] - m);
+            l += p[j];
+        }
+        for (int64_t j = 0; j < n_keys; ++j)
+            p[j] /= l;
+        /* dP row and its P-weighted mean */
+        double pdp = 0.0;
+        for (int64_t j = 0; j < n_keys; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += widen_bf16(doi[c]) * widen_bf16(V[j * d + c]);
+            dp[j] = acc;
+            pdp += p[j] * acc;
+        }
+        for (int64_t j = 0; j < n_keys; ++j) {
+            double ds = p[j] * (dp[j] - pdp);
+            for (int c = 0; c < d; ++c) {
+                dv[j * d + c] += p[j] * widen_bf16(doi[c]);
+                dq[i * d + c] += scale * ds * widen_bf16(K[j * d + c]);
+                dk[j * d + c] += scale * ds * widen_bf16(qi[c]);
+            }
+        }
+    }
+}
+
+typedef struct {
+    const uint16_t *q, *k, *v, *dout;
+    int64_t N;
+    int d, causal;
+    double scale;
+    const int64_t *heads;
+    double *dq, *dk, *dv; /* [nheads, N, d] */
+    int64_t first, last;  /* this thread's share of the head list */
+} bwd_job;
+
+static void *bwd_worker(void *arg)
+{
+    bwd_job *jb = (bwd_job *)arg;
+    const int64_t N = jb->N;
+    const int d = jb->d;
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+    for (int64_t t = jb->first; t < jb->last; ++t) {
+        int64_t off = jb->heads[t] * N * d, out = t * N * d;
+        bwd_head(jb->q + off, jb->k + off, jb->v + off, jb->dout + off, N, d, jb->causal,
+                 jb->scale, jb->dq + out, jb->dk + out, jb->dv + out, p, dp);
+    }
+    free(p);
+    free(dp);
+    return NULL;
+}
+
+/* q, k, v, dout [BH, N, d]; the heads listed in heads[nheads] (indices into BH) are
+ * differentiated; dq, dk, dv [nheads, N, d]. */
+int oracle_attention_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         const uint16_t *dout, int64_t N, int d, int causal, double scale,
+                         const int64_t *heads, int64_t nheads, double *dq, double *dk, double *dv,
+                         int nthreads)
+{
+    if (N < 1 || d < 1 || nheads < 1 || nthreads < 1)
+        return 1;
+    if (nthreads > nheads)
+        nthreads = (int)nheads;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    bwd_job *jobs = (bwd_job *)malloc(sizeof(bwd_job) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) {
+        bwd_job j = {q, k, v, dout, N, d, causal, scale, heads, dq, dk, dv,
+                     nheads * t / nthreads, nheads * (t + 1) / nthreads};
+        jobs[t] = j;
+        pthread_create(&th[t], NULL, bwd_worker, &jobs[t]);
     }
     for (int t = 0; t < nthreads; ++t)
         pthread_join(th[t], NULL);

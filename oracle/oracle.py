@@ -54,8 +54,11 @@ class OracleLib:
                                             _int, _int, _dbl, _f64p, _f64p, _int]
         lib.oracle_prefill_paged.argtypes = [_u16p, _u16p, _u16p, _i32p, _int, _i32p, _int, _int,
                                              _int, _int, _int, _int, _dbl, _f64p, _f64p, _int]
+        lib.oracle_attention_bwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _i64, _int, _int, _dbl,
+                                             _i64p, _i64, _f64p, _f64p, _f64p, _int]
         for f in (lib.oracle_attention, lib.oracle_attention_rows, lib.oracle_attention_probs,
-                  lib.oracle_flash_alg1, lib.oracle_decode_paged, lib.oracle_prefill_paged):
+                  lib.oracle_flash_alg1, lib.oracle_decode_paged, lib.oracle_prefill_paged,
+                  lib.oracle_attention_bwd):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -107,6 +110,28 @@ class OracleLib:
         if rc:
             raise ValueError("oracle_flash_alg1: bad arguments")
         return O, l, m
+
+    def attention_bwd(self, q, k, v, dout, causal: bool, scale: float, heads=None,
+                      nthreads: int | None = None):
+        """Backward pass.  q, k, v, dout: uint16 [..., N, d] (bf16 bits; leading dims flattened to
+        bh).  heads: the bh indices to differentiate (default all).  Returns (dq, dk, dv), each
+        float64 [len(heads), N, d] (or [..., N, d] when all heads are taken)."""
+        q, k, v, dout = _bits(q), _bits(k), _bits(v), _bits(dout)
+        *lead, N, d = q.shape
+        BH = int(np.prod(lead)) if lead else 1
+        all_heads = heads is None
+        heads = np.arange(BH, dtype=np.int64) if all_heads else np.ascontiguousarray(heads, dtype=np.int64)
+        if heads.size and (heads.min() < 0 or heads.max() >= BH):
+            raise ValueError("head index out of range")
+        n = heads.size
+        dq, dk, dv = (np.empty((n, N, d), np.float64) for _ in range(3))
+        rc = self.lib.oracle_attention_bwd(q, k, v, dout, N, d, int(causal), scale, heads, n, dq, dk,
+                                           dv, nthreads or default_threads())
+        if rc:
+            raise ValueError("oracle_attention_bwd: bad arguments")
+        if all_heads:
+            return tuple(t.reshape(*lead, N, d) for t in (dq, dk, dv))
+        return dq, dk, dv
 
     def decode_paged(self, q, k_pool, v_pool, block_table, seq_lens, scale: float, page: int = 16,
                      nthreads: int | None = None):
@@ -185,3 +210,7 @@ def decode_paged(*a, **kw):
 
 def prefill_paged(*a, **kw):
     return default().prefill_paged(*a, **kw)
+
+
+def attention_bwd(*a, **kw):
+    return default().attention_bwd(*a, **kw)

@@ -14,7 +14,12 @@ The facts used:
 * the tiled algorithm of "Flash Attention" (myungum), section 2, computes exact attention, so any
   block sizes give the plain result;
 * a paged KV cache is only a relocation of logically contiguous rows ("LLM study notes", paged
-  attention).
+  attention);
+* the backward pass returns the gradients of sum(dO * O) with respect to Q, K and V (the pages
+  describe it in prose only: "Paged vs Flash attention", training; "Flash Attention" (myungum),
+  section 1, recomputation), so it must agree with central finite differences of the forward
+  definition and with torch.autograd through torch.softmax in fp64, and obey the closed forms that
+  follow from rows of P summing to one and from the shift invariance of the softmax.
 Reference values are formed with numpy/scipy from the widened inputs, never from the oracle.
 """
 from __future__ import annotations
@@ -308,6 +313,86 @@ def pin_paged_prefill(orc):
         close(lse[0, h], lc, 1e-13, "paged prefill Lq=L vs causal attention LSE")
 
 
+def _fwd_loss(Q, K, V, dO, scale, causal):
+    """sum(dO * O) for O = softmax(scale Q K^T, causal) V, fp64 numpy (scipy softmax)."""
+    S_ = scale * Q @ K.T
+    if causal:
+        S_ = np.where(np.tril(np.ones_like(S_, dtype=bool)), S_, -np.inf)
+    return float(np.sum(dO * (sps.softmax(S_, axis=1) @ V)))
+
+
+def pin_bwd_finite_differences(orc):
+    """Every entry of dQ, dK, dV equals the central difference of sum(dO * O) (fp64 forward from
+    scipy's softmax, step 1e-6; truncation ~1e-12, rounding ~1e-10)."""
+    N, d, scale = 6, 4, 0.7
+    q, k, v, do = (rnd((N, d), 90 + t) for t in range(4))
+    Q, K, V, dO = (widen(x) for x in (q, k, v, do))
+    h = 1e-6
+    for causal in (False, True):
+        dq, dk, dv = orc.attention_bwd(q, k, v, do, causal, scale)
+        for name, X, G in (("dQ", Q, dq), ("dK", K, dk), ("dV", V, dv)):
+            fd = np.zeros_like(X)
+            for idx in np.ndindex(*X.shape):
+                Xp, Xm = X.copy(), X.copy()
+                Xp[idx] += h
+                Xm[idx] -= h
+                args_p = [Xp if Y is X else Y for Y in (Q, K, V)]
+                args_m = [Xm if Y is X else Y for Y in (Q, K, V)]
+                fd[idx] = (_fwd_loss(*args_p, dO, scale, causal) -
+                           _fwd_loss(*args_m, dO, scale, causal)) / (2 * h)
+            close(G, fd, 1e-7, f"backward {name} vs finite differences causal={causal}")
+
+
+def pin_bwd_autograd(orc):
+    """dQ, dK, dV equal torch.autograd through torch.softmax in fp64, on two heads of N = 70 (a
+    subset of heads selects the same values)."""
+    B, H, N, d = 1, 2, 70, 16
+    scale = 1.0 / math.sqrt(d)
+    q, k, v, do = (rnd((B, H, N, d), 95 + t) for t in range(4))
+    for causal in (False, True):
+        Q, K, V = (torch.tensor(widen(x), requires_grad=True) for x in (q, k, v))
+        S_ = scale * Q @ K.transpose(-1, -2)
+        if causal:
+            S_ = S_.masked_fill(~torch.ones(N, N, dtype=torch.bool).tril(), float("-inf"))
+        O = torch.softmax(S_, dim=-1) @ V
+        O.backward(torch.tensor(widen(do)))
+        dq, dk, dv = orc.attention_bwd(q, k, v, do, causal, scale)
+        for name, g, t in (("dQ", dq, Q), ("dK", dk, K), ("dV", dv, V)):
+            close(g, t.grad.numpy(), 1e-12, f"backward {name} vs autograd causal={causal}")
+        sq, sk, sv = orc.attention_bwd(q, k, v, do, causal, scale, heads=[1])
+        close(sq[0], dq[0, 1], 0.0, "backward head subset dQ")
+        close(sv[0], dv[0, 1], 0.0, "backward head subset dV")
+
+
+def pin_bwd_closed_forms(orc):
+    """Rows of P sum to one, so sum_j dV_j = sum_i dO_i and each row of dS sums to zero, giving
+    sum_j dK_j = 0.  One key: P = 1, so dQ = dK = 0 and dV = dO.  Q = 0: uniform weights, so every
+    dV_j = mean_i dO_i (non-causal).  Adding one vector u to every key leaves all three gradients
+    unchanged (the softmax ignores a per-row constant)."""
+    N, d, scale = 50, 8, 0.35
+    q, k, v, do = (rnd((N, d), 100 + t) for t in range(4))
+    for causal in (False, True):
+        dq, dk, dv = orc.attention_bwd(q, k, v, do, causal, scale)
+        close(dv.sum(axis=0), widen(do).sum(axis=0), 1e-11, f"sum dV = sum dO causal={causal}")
+        close(dk.sum(axis=0), np.zeros(d), 1e-11, f"sum dK = 0 causal={causal}")
+    q1, k1, v1, do1 = (x[:1].copy() for x in (q, k, v, do))
+    dq, dk, dv = orc.attention_bwd(q1, k1, v1, do1, False, scale)
+    close(dq, np.zeros((1, d)), 0.0, "one key: dQ = 0")
+    close(dk, np.zeros((1, d)), 0.0, "one key: dK = 0")
+    close(dv, widen(do1), 0.0, "one key: dV = dO")
+    dq, dk, dv = orc.attention_bwd(bf16(np.zeros((N, d))), k, v, do, False, scale)
+    close(dv, np.tile(widen(do).mean(axis=0), (N, 1)), 1e-13, "Q = 0: dV_j = mean dO")
+    # keys on a coarse grid so that K + u is exact in bf16
+    kg = bf16(np.round(widen(k) * 4) / 4)
+    ks = bf16(widen(kg) + 0.5 * np.arange(1, d + 1) / d)
+    for causal in (False, True):
+        a = orc.attention_bwd(q, kg, v, do, causal, scale)
+        b = orc.attention_bwd(q, ks, v, do, causal, scale)
+        for name, x, y in zip(("dQ", "dK", "dV"), a, b):
+            close(x, y, 1e-11, f"key shift leaves {name} unchanged causal={causal}")
+
+
 ALL_PINS = [pin_uniform_scores, pin_single_key, pin_dominant_score, pin_two_keys_logistic,
             pin_shift_invariance, pin_rows_sum_to_one, pin_library_softmax, pin_permutation,
-            pin_linear_in_v, pin_tiled_algorithm, pin_paged_decode, pin_paged_prefill]
+            pin_linear_in_v, pin_tiled_algorithm, pin_paged_decode, pin_paged_prefill,
+            pin_bwd_finite_differences, pin_bwd_autograd, pin_bwd_closed_forms]

@@ -38,6 +38,18 @@ MUTANTS = {
                             "int64_t n_keys = jb->causal ? L - Lq + t : L;"),
     "chunk_query_row": ("attend_row(jb->q + r * d, kr, vr, n_keys, d, jb->scale, s, jb->o + r * d, jb->lse + r);",
                         "attend_row(jb->q + (r - t) * d, kr, vr, n_keys, d, jb->scale, s, jb->o + r * d, jb->lse + r);"),
+    "bwd_no_jacobian_mean": ("double ds = p[j] * (dp[j] - pdp);", "double ds = p[j] * dp[j];"),
+    "bwd_dv_weight": ("dv[j * d + c] += p[j] * widen_bf16(doi[c]);",
+                      "dv[j * d + c] += ds * widen_bf16(doi[c]);"),
+    "bwd_dq_scale": ("dq[i * d + c] += scale * ds * widen_bf16(K[j * d + c]);",
+                     "dq[i * d + c] += ds * widen_bf16(K[j * d + c]);"),
+    "bwd_dk_operand": ("dk[j * d + c] += scale * ds * widen_bf16(qi[c]);",
+                       "dk[j * d + c] += scale * ds * widen_bf16(K[j * d + c]);"),
+    "bwd_dp_operand": ("acc += widen_bf16(doi[c]) * widen_bf16(V[j * d + c]);",
+                       "acc += widen_bf16(doi[c]) * widen_bf16(K[j * d + c]);"),
+    "bwd_causal_ignored": ("const int64_t n_keys = causal ? i + 1 : N; /* the keys row i sees */",
+                           "const int64_t n_keys = N;"),
+    "bwd_row_not_normalised": ("            p[j] /= l;\n        /* dP row", "            p[j] /= 1.0;\n        /* dP row"),
 }
 
 
