@@ -15,7 +15,8 @@ Extra keys: `roofline` (prefill kernel vs the measured dense bf16 peak), `cpu_ba
 oracle on this host's cores, a bounded row sample), `e2e` (the same metric through the Python API
 with Q/K/V copied from pinned host memory and O/LSE copied back inside the timed region), `sweep`
 (the sequence-length grid, d = 128 and d = 64), `decode` (paged decode GB/s vs HBM),
-`paged_prefill` (chunked prefill through the block table, TFLOP/s) and `clocks`.
+`paged_prefill` (chunked prefill through the block table, TFLOP/s), `backward` (fa_bwd TFLOP/s)
+and `clocks`.
 """
 from __future__ import annotations
 
@@ -285,6 +286,37 @@ def bench_paged_prefill(fa, args, dev, flush, stream, pk):
             "launches_per_step": 1}
 
 
+def bench_backward(fa, args, dev, flush, stream, pk):
+    """fa_bwd on the headline shape (B8 H16 N2048 d128), non-causal and causal.  FLOPs are the five
+    matmuls per (query, key) pair: 2.5x the forward's 4 B H N^2 d (halved causal)."""
+    out = {}
+    for causal in (False, True):
+        case = W.PrefillCase("bwd", 8, 16, 2048, 128, causal)
+        q, k, v = W.make_prefill(case, device=dev)
+        do = W.make_dout(case, device=dev)
+        o, lse = fa.fa_fwd(q, k, v, causal=causal, scale=case.scale)
+        ws = torch.empty(fa.load_library().fa_bwd_workspace_size(case.B, case.H, case.N, case.d),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: fa.fa_bwd(q, k, v, o, do, lse, causal=causal, scale=case.scale, workspace=ws)
+        torch.cuda.nvtx.range_push("bench_backward_timed")
+        ts = time_launches(fn, args.sweep_steps, 3, flush, stream)
+        torch.cuda.nvtx.range_pop()
+        if fa.device_status() != 0:
+            raise RuntimeError("device status set during the backward bench")
+        ms = statistics.median(ts)
+        tf = 2.5 * case.flops / (ms * 1e-3) / 1e12
+        out["causal" if causal else "non_causal"] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                                                     "frac": round(tf / pk["bf16_tflops"], 4)}
+    tot_ms = out["causal"]["ms"] + out["non_causal"]["ms"]
+    tot_tf = 2.5 * 1.5 * W.PrefillCase("bwd", 8, 16, 2048, 128, False).flops / (tot_ms * 1e-3) / 1e12
+    return {"metric": "attention backward TFLOP/s (dQ, dK, dV; 2.5x forward FLOPs)",
+            "workload": "B8 H16 N2048 d128, dO ~ N(0,1), O and LSE from fa_fwd, causal + non-causal",
+            "value": round(tot_tf, 1), "unit": "TFLOP/s", "per_variant": out,
+            "roofline": {"bound": "tensor", "achieved": round(tot_tf, 1), "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tot_tf / pk["bf16_tflops"], 4)},
+            "launches_per_step": 6}
+
+
 def bench_ours(args, rank, world):
     import exact_attention_158_b200 as fa
     fa.load_library()
@@ -294,6 +326,8 @@ def bench_ours(args, rank, world):
     pk = peaks()
     if args.only == "decode":
         return {"metric": METRIC, "decode": bench_decode(fa, args, dev, flush, stream, pk)}
+    if args.only == "backward":
+        return {"metric": METRIC, "backward": bench_backward(fa, args, dev, flush, stream, pk)}
     if args.only == "paged":
         return {"metric": METRIC,
                 "paged_prefill": bench_paged_prefill(fa, args, dev, flush, stream, pk)}
@@ -415,7 +449,11 @@ def bench_ours(args, rank, world):
     # ---- chunked prefill over the paged cache (tensor bound)
     paged = None if args.no_paged else bench_paged_prefill(fa, args, dev, flush, stream, pk)
 
-    result.update({"e2e": e2e, "sweep": sweep, "decode": dec, "paged_prefill": paged})
+    # ---- backward (tensor bound)
+    bwd = None if args.no_backward else bench_backward(fa, args, dev, flush, stream, pk)
+
+    result.update({"e2e": e2e, "sweep": sweep, "decode": dec, "paged_prefill": paged,
+                   "backward": bwd})
     return result
 
 
@@ -449,10 +487,12 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-paged", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="sequences in the decode workload (64 is the benchmark; fewer for profiling)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "paged"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "paged", "backward"],
+                    default="all",
                     help="prefill: the headline loop alone; decode / paged: the paged decode or "
                     "chunked prefill loop alone")
     args = ap.parse_args()

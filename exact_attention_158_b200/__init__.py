@@ -17,7 +17,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["fa_fwd", "fa_decode_paged", "fa_decode_paged_noalloc", "fa_prefill_paged",
+__all__ = ["fa_fwd", "fa_bwd", "fa_decode_paged", "fa_decode_paged_noalloc", "fa_prefill_paged",
            "fa_decode_workspace_size",
            "NOALLOC_SCRATCH_BYTES", "device_status",
            "FaError", "library_path", "load_library", "EXPORTED_SYMBOLS", "STATUS"]
@@ -27,7 +27,8 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 FA_OUT_BF16, FA_OUT_F32 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
-                    "fa_decode_paged_noalloc", "fa_prefill_paged", "fa_get_device_status",
+                    "fa_decode_paged_noalloc", "fa_prefill_paged", "fa_bwd_workspace_size",
+                    "fa_bwd", "fa_get_device_status",
                     "fa_status_string",
                     "fa_last_error_string", "fa_version", "fa_selftest_wait_timeout")
 
@@ -70,6 +71,11 @@ def load_library():
     lib.fa_prefill_paged.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, i32, vp, i32, i32, i32, i32,
                                      i32, f32, vp]
     lib.fa_prefill_paged.restype = i32
+    lib.fa_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                           f32, vp, ctypes.c_size_t, vp]
+    lib.fa_bwd.restype = i32
     lib.fa_get_device_status.argtypes = [vp]
     lib.fa_get_device_status.restype = i32
     lib.fa_status_string.argtypes = [i32]
@@ -182,6 +188,39 @@ def fa_decode_paged(q, k_pool, v_pool, block_table, seq_lens, scale: float | Non
                                  _stream_handle(stream))
     _check(st, "fa_decode_paged")
     return out, lse
+
+
+def fa_bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = None,
+           grad_dtype=torch.bfloat16, workspace=None, stream=None):
+    """Attention backward: q, k, v, dout bf16 [B, H, N, d]; o (bf16 or fp32) and lse (fp32
+    [B, H, N]) from fa_fwd with the same causal and scale.  Returns (dq, dk, dv) in grad_dtype."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _require(t, n)
+    if o.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError(f"o must be bf16 or fp32, got {o.dtype}")
+    _require(o, "o", o.dtype)
+    _require(lse, "lse", torch.float32)
+    B, H, N, d = q.shape
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        if t.shape != q.shape:
+            raise ValueError(f"{n} must have the shape of q")
+    if lse.shape != (B, H, N):
+        raise ValueError("lse must be [B, H, N]")
+    code = _out_code(grad_dtype)
+    need = int(lib.fa_bwd_workspace_size(B, H, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = (torch.empty(q.shape, dtype=grad_dtype, device=q.device) for _ in range(3))
+    with torch.cuda.device(q.device):
+        st = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _out_code(o.dtype),
+                        dout.data_ptr(),
+                        lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), code, B, H, N,
+                        d, int(causal), float(scale) if scale is not None else 0.0,
+                        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                        _stream_handle(stream))
+    _check(st, "fa_bwd")
+    return dq, dk, dv
 
 
 def fa_prefill_paged(q, k_pool, v_pool, block_table, seq_lens, causal: bool = True,

@@ -1,6 +1,6 @@
 // fa_lib.cu -- the C ABI declared in include/fa.h: argument checks, TMA descriptors, launches.
 // Host code only decides shapes and launches; every step of the attention itself runs in the
-// kernels of fa_prefill.cuh and fa_decode.cuh.
+// kernels of fa_prefill.cuh, fa_backward.cuh and fa_decode.cuh.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -13,6 +13,7 @@
 #include <string>
 
 #include "fa.h"
+#include "fa_backward.cuh"
 #include "fa_decode.cuh"
 #include "fa_prefill.cuh"
 
@@ -46,6 +47,7 @@ struct DeviceInfo {
   bool supported = false;
   int num_sms = 0;
   bool prefill_attr[4] = {false, false, false, false};  // (d = 64, 128) x (contiguous, paged)
+  bool bwd_attr[2] = {false, false};                    // d = 64, 128
 };
 
 std::mutex g_mutex;
@@ -180,6 +182,75 @@ fa_status launch_prefill_dense(DeviceInfo &dev, const void *q, const void *k, co
   return launch_prefill<HD, false>(dev, tq, tk, tv, p, stream);
 }
 
+// Backward workspace: dQ accumulator fp32 [BH, Np, d], then LSE2 and D fp32 [BH, Np] each, with
+// Np = N rounded up to the 128-row block.
+size_t bwd_padded_rows(int BH, int N) {
+  return static_cast<size_t>(BH) * ((static_cast<size_t>(N) + fa::kBM - 1) / fa::kBM * fa::kBM);
+}
+
+template <int HD>
+fa_status launch_bwd(DeviceInfo &dev, const void *q, const void *k, const void *v, const void *o,
+                     int o_f32, const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                     int g_f32,
+                     int BH, int N, int causal, float scale, void *workspace, cudaStream_t stream) {
+  using C = fa::BwdCfg<HD>;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bhnd(&tq, q, HD, N, BH) || !encode_bhnd(&tk, k, HD, N, BH) ||
+      !encode_bhnd(&tv, v, HD, N, BH) || !encode_bhnd(&tdo, dout, HD, N, BH)) {
+    t_last_error = "cuTensorMapEncodeTiled failed";
+    return FA_ERR_LAUNCH;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!dev.bwd_attr[HD == 128]) {
+      cudaError_t e = cudaFuncSetAttribute(fa::fa_bwd_kernel<HD>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(C::kSmemBytes));
+      if (e != cudaSuccess) return launch_failed(e);
+      dev.bwd_attr[HD == 128] = true;
+    }
+  }
+  const int Np = (N + fa::kBM - 1) / fa::kBM * fa::kBM;
+  const size_t prow = static_cast<size_t>(BH) * Np;
+  float *dq_acc = static_cast<float *>(workspace);
+  float *lse2 = dq_acc + prow * HD;
+  float *dvec = lse2 + prow;
+  constexpr int kRowThreads = HD / 8;
+  const long long prep_threads = static_cast<long long>(prow) * kRowThreads;
+  const unsigned prep_blocks = static_cast<unsigned>((prep_threads + 255) / 256);
+  if (o_f32)
+    fa::fa_bwd_prep_kernel<HD, true><<<prep_blocks, 256, 0, stream>>>(
+        o, static_cast<const uint16_t *>(dout), lse, lse2, dvec, dq_acc, BH, N, Np);
+  else
+    fa::fa_bwd_prep_kernel<HD, false><<<prep_blocks, 256, 0, stream>>>(
+        o, static_cast<const uint16_t *>(dout), lse, lse2, dvec, dq_acc, BH, N, Np);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return launch_failed(e);
+  fa::BwdParams p{};
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.dq_acc = dq_acc;
+  p.dk = dk;
+  p.dv = dv;
+  p.g_f32 = g_f32;
+  p.BH = BH;
+  p.N = N;
+  p.Np = Np;
+  p.nkb = Np / fa::kBN;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  const long long units = static_cast<long long>(BH) * p.nkb;
+  fa::fa_bwd_kernel<HD><<<static_cast<unsigned>(units), fa::kBwdThreads, C::kSmemBytes, stream>>>(
+      tq, tk, tv, tdo, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return launch_failed(e);
+  const long long post_threads = static_cast<long long>(BH) * N * kRowThreads;
+  fa::fa_bwd_dq_kernel<HD><<<static_cast<unsigned>((post_threads + 255) / 256), 256, 0, stream>>>(
+      dq_acc, dq, g_f32, scale, BH, N, Np);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : launch_failed(e);
+}
+
 int decode_splits(int max_blocks) {
   return (max_blocks + fa::kDecodeChunkPages - 1) / fa::kDecodeChunkPages;
 }
@@ -219,6 +290,60 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, fa_out_dt
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128) return launch_prefill_dense<128>(*dev, q, k, v, o, o_f32, lse, BH, N, causal, sc, s);
   return launch_prefill_dense<64>(*dev, q, k, v, o, o_f32, lse, BH, N, causal, sc, s);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  if (static_cast<long long>(B) * H > INT_MAX) return 0;
+  return bwd_padded_rows(B * H, N) * (d + 2) * sizeof(float);
+}
+
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, fa_out_dtype o_dtype,
+                 const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                 fa_out_dtype g_dtype, int B, int H, int N, int d, int causal, float scale,
+                 void *workspace, size_t workspace_bytes, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (g_dtype != FA_OUT_BF16 && g_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  const int BH = B * H;
+  if (static_cast<long long>(BH) * ((N + fa::kBN - 1) / fa::kBN) > INT_MAX) return FA_ERR_INVALID_ARG;
+  float sc;
+  if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_ALIGNMENT;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
+  const size_t rows = static_cast<size_t>(BH) * N;
+  const size_t in_bytes = rows * d * 2, g_bytes = rows * d * (g_dtype == FA_OUT_F32 ? 4 : 2);
+  const size_t o_bytes = rows * d * (o_dtype == FA_OUT_F32 ? 4 : 2);
+  const void *ins[6] = {q, k, v, o, dout, lse};
+  const size_t in_sizes[6] = {in_bytes, in_bytes, in_bytes, o_bytes, in_bytes, rows * 4};
+  void *outs[4] = {dq, dk, dv, workspace};
+  const size_t out_sizes[4] = {g_bytes, g_bytes, g_bytes, need};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps(outs[a], out_sizes[a], ins[b], in_sizes[b])) return FA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], out_sizes[a], outs[b], out_sizes[b])) return FA_ERR_INVALID_ARG;
+  }
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  const int g_f32 = g_dtype == FA_OUT_F32, o_f32 = o_dtype == FA_OUT_F32;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return launch_bwd<128>(*dev, q, k, v, o, o_f32, dout, lse, dq, dk, dv, g_f32, BH, N, causal,
+                           sc, workspace, s);
+  return launch_bwd<64>(*dev, q, k, v, o, o_f32, dout, lse, dq, dk, dv, g_f32, BH, N, causal, sc,
+                        workspace, s);
 }
 
 size_t fa_decode_workspace_size(int num_seqs, int H, int d, int max_blocks_per_seq) {

@@ -1,7 +1,7 @@
 /*
  * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa_b200.so).
  *
- * Operation.  Exact scaled-dot-product attention, forward only:
+ * Operation.  Exact scaled-dot-product attention (forward, and its backward in fa_bwd):
  *     O = softmax(scale * Q K^T [+ causal mask]) V,   LSE_i = log sum_j exp(scale * q_i . k_j)
  * computed tile by tile with a running row max and row sum, so the N x N score matrix never
  * leaves the chip ("Flash Attention" (velog.io/@myungum), section 2 and its pseudocode: blocks of
@@ -73,6 +73,42 @@ typedef enum {
 fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, fa_out_dtype o_dtype,
                  float *lse, int B, int H, int N, int d, int causal, float scale,
                  fa_stream_t stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs: 4 * (d + 2) per query row, with
+ * N rounded up to a multiple of 128.  Returns 0 on invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd -- attention backward: the gradients dQ, dK, dV of sum(dO * O) for O = fa_fwd(q, k, v).
+ *
+ * The pages give the backward in prose only: gradients are computed block by block from the
+ * intermediate results the forward kept ("Paged vs Flash attention", training), and the attention
+ * matrix is recomputed rather than stored ("LLM study notes", FlashAttention; "Flash Attention"
+ * (myungum), section 1).  The forward keeps LSE; P is recomputed tile by tile as
+ * exp(scale q.k - LSE), and with D_i = sum_c dO[i,c] O[i,c]:
+ *     dV = P^T dO,  dS = P * (dO V^T - D),  dQ = scale dS K,  dK = scale dS^T Q.
+ *
+ *   q, k, v, dout     bf16 [B, H, N, d] contiguous, 16-byte aligned; dout is the incoming gradient.
+ *   o, o_dtype        fa_fwd's output for the same q, k, v, causal and scale, [B, H, N, d] in bf16
+ *                     or fp32.  D is formed from it, so bf16 O carries its own rounding (2^-9
+ *                     relative) into dS; fp32 O avoids that where rows are nearly one-hot.
+ *   lse               fp32 [B, H, N], fa_fwd's log-sum-exp for the same call.
+ *   dq, dk, dv        [B, H, N, d], bf16 or fp32 per g_dtype, 16-byte aligned; must not overlap the
+ *                     inputs, one another or the workspace.
+ *   B, H, N, d, causal, scale   as for fa_fwd.
+ *   workspace         device scratch of at least fa_bwd_workspace_size(B, H, N, d) bytes, 16-byte
+ *                     aligned, owned by the caller; no initialisation needed, garbage afterwards.
+ *                     Two calls in flight at once need separate workspaces.
+ * Three kernels are queued on the stream (row statistics, the blockwise gradients, the dQ
+ * conversion).  dQ is summed in fp32 with atomic adds, so its last bits may differ between runs;
+ * dK and dV are deterministic.  Returns FA_OK once the kernels are queued.
+ */
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, fa_out_dtype o_dtype,
+                 const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                 fa_out_dtype g_dtype, int B, int H, int N, int d, int causal, float scale,
+                 void *workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fa_decode_workspace_size -- bytes of device workspace fa_decode_paged needs for these sizes.

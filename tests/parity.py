@@ -90,3 +90,66 @@ def run_prefill(case: W.PrefillCase, out_dtype=torch.float32, full: bool | None 
     lg = lse.reshape(BH, N)[pairs[:, 0], pairs[:, 1]].cpu().numpy()
     return assert_close(og, lg, o_ref, lse_ref, case.name + " (sampled rows)",
                         out_bf16=out_dtype == torch.bfloat16)
+
+
+# Backward tolerance.  Each gradient is an fp32 sum of products whose device-formed factor passed
+# through bf16 (unit roundoff u = 2^-9): P for dV, and P then dS = P (dP - D) for dK and dQ, with D
+# itself formed from the bf16 forward output.  Two roundings of 2^-9 and a cancellation factor of
+# up to 4 in the sums give 2^-6 of the tensor's largest magnitude for the worst element, and 2^-7 of
+# its mean magnitude on average; 2^-16 absolute covers tensors that are exactly zero (one key).
+TOL_GRAD_MAX = 2.0 ** -6
+TOL_GRAD_MEAN = 2.0 ** -7
+TOL_GRAD_ABS = 2.0 ** -16
+
+
+def assert_grads_close(got, ref, what="", out_bf16=False):
+    """got, ref: dicts name -> array (same shapes).  Per tensor: max|d| <= 2^-6 max|ref| + 2^-16 and
+    mean|d| <= 2^-7 mean|ref| + 2^-16; bf16 gradients add their own rounding (2^-8 |ref| per
+    element, 2^-9 on average)."""
+    out = {}
+    for name in ref:
+        g = np.asarray(got[name], np.float64)
+        r = np.asarray(ref[name], np.float64)
+        assert g.shape == r.shape, f"{what} {name}: shape {g.shape} vs {r.shape}"
+        assert np.all(np.isfinite(g)), f"{what} {name}: non-finite gradient"
+        d = np.abs(g - r)
+        if out_bf16:
+            d = np.maximum(d - BF16_REL * np.abs(r), 0.0)
+        mx, mean = float(d.max()), float(d.mean())
+        lim_max = TOL_GRAD_MAX * float(np.abs(r).max()) + TOL_GRAD_ABS
+        lim_mean = TOL_GRAD_MEAN * float(np.abs(r).mean()) + TOL_GRAD_ABS
+        log = os.environ.get("FA_PARITY_LOG")
+        if log:
+            with open(log, "a") as f:
+                f.write(json.dumps({"case": f"{what} {name}", "out": "bf16" if out_bf16 else "f32",
+                                    "max_err": mx, "lim_max": lim_max, "mean_err": mean,
+                                    "lim_mean": lim_mean, "n": int(d.size)}) + "\n")
+        assert mx <= lim_max, f"{what} {name}: max err {mx:.3e} > {lim_max:.3e}"
+        assert mean <= lim_mean, f"{what} {name}: mean err {mean:.3e} > {lim_mean:.3e}"
+        out[name] = (mx, mean)
+    return out
+
+
+def run_backward(case: W.PrefillCase, grad_dtype=torch.float32, heads=None, scale=None,
+                 o_dtype=torch.bfloat16):
+    """fa_fwd (O in o_dtype) then fa_bwd on the case (dO from the shared generator); the listed
+    heads (default all) compared with the oracle's backward.  scale: override of 1/sqrt(d)."""
+    scale = case.scale if scale is None else scale
+    import exact_attention_158_b200 as fa
+    q, k, v = W.make_prefill(case, device="cuda")
+    do = W.make_dout(case, device="cuda")
+    o, lse = fa.fa_fwd(q, k, v, causal=case.causal, scale=scale, out_dtype=o_dtype)
+    dq, dk, dv = fa.fa_bwd(q, k, v, o, do, lse, causal=case.causal, scale=scale,
+                           grad_dtype=grad_dtype)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    BH, N, d = case.B * case.H, case.N, case.d
+    if heads is None:
+        heads = list(range(BH))
+    rq, rk, rv = orc.attention_bwd(*(W.bf16_bits(t).reshape(BH, N, d) for t in (q, k, v, do)),
+                                   case.causal, scale, heads=heads)
+    pick = lambda t: t.float().reshape(BH, N, d)[heads].cpu().numpy()
+    return assert_grads_close({"dq": pick(dq), "dk": pick(dk), "dv": pick(dv)},
+                              {"dq": rq, "dk": rk, "dv": rv},
+                              f"{case.name} o={'f32' if o_dtype == torch.float32 else 'bf16'}",
+                              out_bf16=grad_dtype == torch.bfloat16)

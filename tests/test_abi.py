@@ -100,6 +100,27 @@ def test_prefill_paged_rejections(lib):
     assert pp(lib, o=2 * A + 64) == 1  # output overlaps the K pool
 
 
+def bwd(lib, dq=8 * A, ws=12 * A, ws_bytes=1 << 30, B=1, H=2, N=300, d=128, causal=0, dt=0,
+        lse=6 * A, scale=0.0, odt=0):
+    return lib.fa_bwd(A, 2 * A, 3 * A, 4 * A, odt, 5 * A, lse, dq, 9 * A, 10 * A, dt, B, H, N, d,
+                      causal, scale, ws, ws_bytes, None)
+
+
+def test_bwd_workspace_and_rejections(lib):
+    # N = 300 pads to 384 rows: dQ accumulator (d floats) + LSE2 + D per row
+    assert lib.fa_bwd_workspace_size(1, 2, 300, 128) == 2 * 384 * (128 + 2) * 4
+    assert lib.fa_bwd_workspace_size(1, 2, 300, 80) == 0
+    assert lib.fa_bwd_workspace_size(0, 2, 300, 64) == 0
+    assert bwd(lib, ws=None) == 6 and bwd(lib, ws_bytes=1000) == 6
+    assert bwd(lib, B=0) == 1 and bwd(lib, N=0) == 1 and bwd(lib, causal=5) == 1
+    assert bwd(lib, dt=3) == 1 and bwd(lib, lse=None) == 1 and bwd(lib, odt=2) == 1
+    assert bwd(lib, d=32) == 2
+    assert bwd(lib, dq=8 * A + 8) == 3 and bwd(lib, lse=6 * A + 2) == 3 and bwd(lib, ws=12 * A + 4) == 3
+    assert bwd(lib, dq=A + 1024) == 1   # dQ overlaps q
+    assert bwd(lib, dq=9 * A + 64) == 1  # dQ overlaps dK
+    assert bwd(lib, ws=10 * A + 64) == 1  # workspace overlaps dV
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)

@@ -30,7 +30,7 @@ from dataclasses import dataclass, field
 import torch
 
 BASE_SEED = 158
-TID_Q, TID_K, TID_V, TID_LENS, TID_PERM, TID_PEAKS = 1, 2, 3, 4, 5, 6
+TID_Q, TID_K, TID_V, TID_LENS, TID_PERM, TID_PEAKS, TID_DO = 1, 2, 3, 4, 5, 6, 7
 PAGE_SIZE = 16
 
 _M64 = (1 << 64) - 1
@@ -218,6 +218,12 @@ class DecodeCase:
         if self.lens is not None:
             return list(self.lens)
         return uniform_ints(self.seed, TID_LENS, self.S, self.len_lo, self.len_hi)
+
+
+def make_dout(case: PrefillCase, device="cpu"):
+    """The incoming gradient dO for the backward pass: bf16 [B, H, N, d], i.i.d. N(0, 1)."""
+    shape = (case.B, case.H, case.N, case.d)
+    return normal_bf16(case.seed, TID_DO, case.B * case.H * case.N * case.d, device).view(shape)
 
 
 def make_decode(case: DecodeCase, device="cpu"):
