@@ -18,21 +18,26 @@
 // The scores are computed transposed, S^T = K_j Q_i^T (TMEM lane = key), so each compute thread
 // owns one key row: P^T and dS^T are written by rows into one 128 x 128 bf16 tile X in the
 // 128-byte-swizzled layout the tensor core reads.  X is the K-major A operand of dV += P^T dO and
-// dK += dS^T Q, and, read through an MN-major descriptor, the A operand of dQ = dS K.
+// dK += dS^T Q, and, read through MN-major descriptors, an operand of the dQ product.  At d = 128
+// that product is dQ^T = K_j^T dS^T (TMEM lane = feature), so the read-out adds 32 consecutive
+// floats of one dQ row per warp instruction; at d = 64 it is dQ = dS K_j (lane = query).
 //
-//   warps 0-3  compute: S^T -> P^T (X), dP^T -> dS^T (X), and the final dK, dV write
-//   warps 4-7  dQ: TMEM -> fp32 red.add into the accumulator
-//   warp  8    TMA producer: K_j, V_j once; Q_i (+ its LSE and D rows), dO_i per query block
-//   warp  9    MMA issuer (one thread) + TMEM owner
-// TMEM (512 columns): S^T [0,128)  dP^T [128,256)  dV [256,256+d)  dK [256+d,256+2d)  and dQ at
-// [256+2d, 256+3d) when d = 64; at d = 128 the columns are full and dQ_i takes dP^T's columns,
-// which are free once dS^T_i has been formed.
+//   warps 0-3, 4-7  compute, one key row per thread, query columns [0,64) and [64,128): P^T and
+//                   dS^T, and the final dK, dV write
+//   warps 8-11      dQ read-out: TMEM -> a shared-memory staging box -> a bulk tensor reduction
+//                   (fp32 add) into the accumulator, one box of 32 features per warp at a time
+//   warp  12        TMA producer: K_j, V_j once; Q_i (+ its LSE and D rows), dO_i per query block
+//   warp  13        MMA issuer (one thread) + TMEM owner
+// TMEM (512 columns): S^T [0,128)  dP^T [128,256)  dV [256,256+d)  dK [256+d,256+2d); dQ at
+// [256+2d, 256+3d) when d = 64, and in S^T's columns when d = 128 (they are full otherwise).
+// MMA order per query block t: dV_t, S^T_t+1, dK_t, dQ_t, dP^T_t+1 -- so that the tensor core has
+// the next block's products queued while the compute warps turn S^T into P^T and dP^T into dS^T.
 #pragma once
 #include "fa_prefill.cuh"
 
 namespace fa {
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 448;
 constexpr size_t kMaxDynSmem = 232448;  // 227 KB per CTA on sm_100
 
 template <int HD>
@@ -42,23 +47,31 @@ struct BwdCfg {
   static constexpr int kChunkBytes = 128 * 128;
   static constexpr int kTileBytes = 128 * HD * 2;
   static constexpr int kXBytes = 128 * 128 * 2;
-  static constexpr int kStages = 2;                // Q and dO rings
+  static constexpr int kStages = 2;                // Q ring
+  static constexpr int kDoStages = HD == 128 ? 1 : 2;  // dO ring (one stage frees room at d = 128)
+  // dQ staging: one 8 KB slot per read-out warp, boxes of 32 features x kBoxRows rows, fp32,
+  // 128-byte swizzle (d = 128: 64 query rows; d = 64: the warp's 32 query rows)
+  static constexpr int kBoxRows = HD == 128 ? 64 : 32;
+  static constexpr int kStageSlotBytes = 8192;
   static constexpr int kVecFloats = 2 * kBM;       // LSE (log2 units) and D of one query block
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + HD;
-  static constexpr bool kDqOnDp = HD == 128;
-  static constexpr uint32_t kColDQ = kDqOnDp ? kColDP : 256 + 2 * HD;
+  static constexpr bool kDqT = HD == 128;          // dQ^T in S^T's columns (lane = feature)
+  static constexpr uint32_t kColDQ = kDqT ? kColS : 256 + 2 * HD;
   static constexpr int kTmemCols = 512;
-  static constexpr int kNumBars = 1 + 4 * kStages + 10;
-  static constexpr size_t kBodyBytes = 2 * kTileBytes + 2 * kStages * kTileBytes + kXBytes +
-                                       kStages * kVecFloats * 4 + kNumBars * 8 + 16;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 * kDoStages + 9;
+  static constexpr size_t kBodyBytes = 2 * kTileBytes + (kStages + kDoStages) * kTileBytes +
+                                       kXBytes + 4 * kStageSlotBytes + kStages * kVecFloats * 4 +
+                                       kNumBars * 8 + 16;
   // up to 1 KB of slack to align the tiles to the 1024-byte swizzle atom
   static constexpr size_t kSmemBytes =
       kBodyBytes + 1024 <= kMaxDynSmem ? kBodyBytes + 1024 : kMaxDynSmem;
   static_assert(kBodyBytes <= kMaxDynSmem, "shared memory budget");
-  static_assert(kColDQ + (kDqOnDp ? 0 : HD) <= kTmemCols, "TMEM budget");
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);  // K/V and Q/dO K-major
+  static_assert(kColDQ + (kDqT ? 0 : HD) <= kTmemCols, "TMEM budget");
   static constexpr uint32_t kIdescKV = idesc_bf16_f32(128, HD, 0, 1);  // X K-major, Q/dO MN-major
-  static constexpr uint32_t kIdescQ = idesc_bf16_f32(128, HD, 1, 1);   // X MN-major, K MN-major
+  // dQ^T (d = 128): A = K^T MN-major (m = feature), B = dS^T MN-major (n = query);
+  // dQ (d = 64): A = dS MN-major (m = query), B = K MN-major (n = feature)
+  static constexpr uint32_t kIdescQ = kDqT ? idesc_bf16_f32(HD, 128, 1, 1)
+                                           : idesc_bf16_f32(128, HD, 1, 1);
 };
 
 struct BwdParams {
@@ -84,25 +97,37 @@ __device__ __forceinline__ void issue_x_kmajor(uint32_t d_tmem, uint32_t x_smem,
   }
 }
 
-// dQ (TMEM, 128 queries x HD) = dS K: A = X read MN-major (m = query = X's column, k = key = X's
-// row), B = K_j read MN-major (n = d, k = key).
+// The dQ product over the 128 keys of the block, both operands MN-major with the key as K:
+// d = 128: dQ^T = K^T dS^T (A from the K tile, B from X); d = 64: dQ = dS K (A from X, B from K).
 template <int HD>
 __device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t x_smem, uint32_t k_smem) {
   using C = BwdCfg<HD>;
+  const uint32_t a_base = C::kDqT ? k_smem : x_smem, b_base = C::kDqT ? x_smem : k_smem;
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk) {
-    const uint64_t a = smem_desc_sw128(x_smem + kk * 16 * 128, 16384, 1024);
-    const uint64_t b = smem_desc_sw128(k_smem + kk * 16 * 128, 16384, 1024);
+    const uint64_t a = smem_desc_sw128(a_base + kk * 16 * 128, 16384, 1024);
+    const uint64_t b = smem_desc_sw128(b_base + kk * 16 * 128, 16384, 1024);
     umma_ss(d_tmem, a, b, C::kIdescQ, kk > 0 ? 1u : 0u);
   }
 }
 
-// One TMEM row of HD fp32 values (this thread's lane) times `mul`, to global row `grow`.
-template <int HD>
-__device__ __forceinline__ void store_grad_row(uint32_t taddr, float mul, void *dst_base, int f32,
-                                               size_t grow, bool live) {
+// Half a row of X (this thread's key row r, query columns [64 h, 64 h + 64) = swizzle chunk h):
+// 32 packed bf16 pairs, the 16-byte unit u stored at unit u ^ (r % 8).
+__device__ __forceinline__ void store_x_half(uint8_t *x_tile, int r, int h, const uint32_t (&pk)[32]) {
+  uint8_t *rowp = x_tile + h * 16384 + r * 128;
 #pragma unroll
-  for (int cc = 0; cc < HD; cc += 32) {
+  for (int u = 0; u < 8; ++u)
+    *reinterpret_cast<uint4 *>(rowp + ((u ^ (r & 7)) * 16)) =
+        make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+}
+
+// Columns [c0, c0 + 32 * NCH) of this thread's TMEM row, times `mul`, to global row `grow`.
+template <int HD, int NCH>
+__device__ __forceinline__ void store_grad_cols(uint32_t taddr, int c0, float mul, void *dst_base,
+                                                int f32, size_t grow, bool live) {
+#pragma unroll
+  for (int ch = 0; ch < NCH; ++ch) {
+    const int cc = c0 + 32 * ch;
     uint32_t v[32];
     tmem_ld32(taddr + cc, v);
     tmem_wait_ld();
@@ -128,11 +153,78 @@ __device__ __forceinline__ void store_grad_row(uint32_t taddr, float mul, void *
   }
 }
 
+// Add dQ_i's partial (TMEM) into the accumulator through this read-out warp's staging slot.
+// Warp w (0..3) reads TMEM lanes 32 w .. 32 w + 31 and owns the boxes those lanes fill:
+//   d = 128 (dQ^T, lane = feature f = 32 w + lane): two boxes of 64 query rows x 32 features; each
+//           query column of TMEM becomes one 128-byte row of the box (one 4-byte store per lane).
+//   d = 64  (dQ, lane = query 32 w + lane): two boxes of the warp's 32 query rows x 32 features;
+//           each thread stores its row (8 x 16 bytes).
+// Stores use the 128-byte swizzle of the tensor map (16-byte unit u of row r at u ^ (r % 8)).
+// The dQ columns are released (dq_free) as soon as TMEM has been read; the slot is reused once the
+// bulk reduction has finished reading it.
+template <int HD>
+__device__ __forceinline__ void read_out_dq(uint32_t tq, int w, int lane, uint8_t *slot,
+                                            const CUtensorMap *tm_dq, int row0, uint64_t *dq_free) {
+  using C = BwdCfg<HD>;
+  if constexpr (C::kDqT) {
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      uint32_t v[2][32];
+      tmem_ld32(tq + 64 * half, v[0]);
+      tmem_ld32(tq + 64 * half + 32, v[1]);
+      tmem_wait_ld();
+      if (half == 1) {  // TMEM fully read: the columns may take the next block's S^T
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free);
+      }
+      if (lane == 0) bulk_wait_group_read<0>();  // the previous box has left the slot
+      __syncwarp();
+      const int unit = lane / 4, sub = (lane % 4) * 4;
+#pragma unroll
+      for (int q = 0; q < 64; ++q)
+        *reinterpret_cast<float *>(slot + q * 128 + ((unit ^ (q & 7)) * 16) + sub) =
+            __uint_as_float(v[q / 32][q % 32]);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_2d(tm_dq, slot, 32 * w, row0 + 64 * half);
+        bulk_commit_group();
+      }
+    }
+  } else {
+    uint32_t v[2][32];
+    tmem_ld32(tq, v[0]);
+    tmem_ld32(tq + 32, v[1]);
+    tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(dq_free);
+    if (lane == 0) bulk_wait_group_read<0>();
+    __syncwarp();
+#pragma unroll
+    for (int fg = 0; fg < 2; ++fg) {
+      uint8_t *rowp = slot + fg * 4096 + lane * 128;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4 *>(rowp + ((u ^ (lane & 7)) * 16)) =
+            make_uint4(v[fg][4 * u], v[fg][4 * u + 1], v[fg][4 * u + 2], v[fg][4 * u + 3]);
+    }
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_reduce_add_2d(tm_dq, slot, 0, row0 + 32 * w);
+      tma_reduce_add_2d(tm_dq, slot + 4096, 32, row0 + 32 * w);
+      bulk_commit_group();
+    }
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
@@ -144,23 +236,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t *sK = reinterpret_cast<uint8_t *>(base);
   uint8_t *sV = sK + C::kTileBytes;
   uint8_t *sQ = sV + C::kTileBytes;                 // kStages tiles
-  uint8_t *sDO = sQ + C::kStages * C::kTileBytes;   // kStages tiles
-  uint8_t *sX = sDO + C::kStages * C::kTileBytes;   // P^T, then dS^T
-  float *sVec = reinterpret_cast<float *>(sX + C::kXBytes);  // [kStages][LSE2 128 | D 128]
+  uint8_t *sDO = sQ + C::kStages * C::kTileBytes;   // kDoStages tiles
+  uint8_t *sX = sDO + C::kDoStages * C::kTileBytes; // P^T, then dS^T
+  uint8_t *sStage = sX + C::kXBytes;                // 4 dQ staging slots
+  float *sVec = reinterpret_cast<float *>(sStage + 4 * C::kStageSlotBytes);  // [kStages][LSE2 | D]
   uint64_t *bars = reinterpret_cast<uint64_t *>(sVec + C::kStages * C::kVecFloats);
   uint64_t *kv_full = bars;                    // K_j, V_j landed
   uint64_t *q_full = bars + 1;                 // [kStages] Q_i + its LSE2 / D rows landed
   uint64_t *q_empty = q_full + C::kStages;     // [kStages] dK_i done (last reader of Q_i)
-  uint64_t *do_full = q_empty + C::kStages;    // [kStages] dO_i landed
-  uint64_t *do_empty = do_full + C::kStages;   // [kStages] dV_i done (last reader of dO_i)
-  uint64_t *s_full = do_empty + C::kStages;    // S^T_i computed
-  uint64_t *s_free = s_full + 1;               // S^T_i copied out (4 warp arrivals)
+  uint64_t *do_full = q_empty + C::kStages;    // [kDoStages] dO_i landed
+  uint64_t *do_empty = do_full + C::kDoStages; // [kDoStages] dV_i done (last reader of dO_i)
+  uint64_t *s_full = do_empty + C::kDoStages;  // S^T_i computed
+  uint64_t *s_free = s_full + 1;               // S^T_i copied out (8 warp arrivals)
   uint64_t *dp_full = s_free + 1;              // dP^T_i computed
-  uint64_t *p_full = dp_full + 1;              // P^T_i written to X (4 warp arrivals)
+  uint64_t *p_full = dp_full + 1;              // P^T_i written to X (8 warp arrivals)
   uint64_t *dv_done = p_full + 1;              // dV += P^T_i dO_i done: X may take dS^T_i
-  uint64_t *ds_full = dv_done + 1;             // dS^T_i written to X (4 warp arrivals)
-  uint64_t *x_free = ds_full + 1;              // dK_i and dQ_i done: X may take P^T_i+1
-  uint64_t *dq_full = x_free + 1;              // dQ_i computed
+  uint64_t *ds_full = dv_done + 1;             // dS^T_i written to X (8 warp arrivals)
+  uint64_t *dq_full = ds_full + 1;             // dK_i and dQ_i done: dQ_i readable, X free
   uint64_t *dq_free = dq_full + 1;             // dQ_i read out (4 warp arrivals)
   uint64_t *drain = dq_free + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -172,44 +264,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int bh = blockIdx.x / p.nkb;
   const int i_lo = p.causal ? jb : 0;  // first query block that sees key block jb
   const int n = p.Np / kBM - i_lo;     // query blocks visited (>= 1)
+  // Visit order: step t takes query block i_lo + (t + rot) mod n.  The CTAs of one head run at the
+  // same time and all add into that head's dQ; starting each key block's loop at a different
+  // query block (rot = jb without the mask; with it, i_lo = jb already staggers them) keeps them
+  // from reducing into the same dQ rows at the same moment.
+  const int rot = p.causal ? 0 : jb % n;
+  auto qblock = [&](int t) { return i_lo + (t + rot) % n; };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < C::kDoStages; ++s) {
       mbar_init(&do_full[s], 1);
       mbar_init(&do_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
+    mbar_init(s_free, 8);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(dv_done, 1);
-    mbar_init(ds_full, 4);
-    mbar_init(x_free, 1);
+    mbar_init(ds_full, 8);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
@@ -221,7 +321,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const size_t vec_row = static_cast<size_t>(bh) * p.Np;
       for (int t = 0; t < n; ++t) {
-        const int i = i_lo + t, st = t % C::kStages;
+        const int i = qblock(t), st = t % C::kStages;
         const uint32_t ph = (t / C::kStages) & 1;
         if (!mbar_wait(&q_empty[st], ph ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(&q_full[st], C::kTileBytes + C::kVecFloats * 4);
@@ -232,10 +332,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bulk_load_1d(vec, p.lse2 + vec_row + i * kBM, kBM * 4, &q_full[st]);
         bulk_load_1d(vec + kBM, p.dvec + vec_row + i * kBM, kBM * 4, &q_full[st]);
         ++q_loads;
-        if (!mbar_wait(&do_empty[st], ph ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&do_full[st], C::kTileBytes);
+        const int sd = t % C::kDoStages;
+        if (!mbar_wait(&do_empty[sd], ((t / C::kDoStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&do_full[sd], C::kTileBytes);
         for (int ch = 0; ch < C::kChunks; ++ch)
-          tma_load_3d(sDO + st * C::kTileBytes + ch * C::kChunkBytes, &tm_do, &do_full[st],
+          tma_load_3d(sDO + sd * C::kTileBytes + ch * C::kChunkBytes, &tm_do, &do_full[sd],
                       ch * 64, i * kBM, bh);
         ++do_loads;
       }
@@ -245,54 +346,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_wait(kv_full, 0, &never);
         for (int t = q_loads - C::kStages; t < q_loads; ++t)
           if (t >= 0) mbar_wait(&q_full[t % C::kStages], (t / C::kStages) & 1, &never);
-        for (int t = do_loads - C::kStages; t < do_loads; ++t)
-          if (t >= 0) mbar_wait(&do_full[t % C::kStages], (t / C::kStages) & 1, &never);
+        for (int t = do_loads - C::kDoStages; t < do_loads; ++t)
+          if (t >= 0) mbar_wait(&do_full[t % C::kDoStages], (t / C::kDoStages) & 1, &never);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------------ MMA issuer
-    // Per query block t: S^T_t+1 as soon as the compute warps have copied S^T_t out, then
-    // dV += P^T_t dO_t, dK += dS^T_t Q_t, dQ_t = dS_t K, then dP^T_t+1.
     if (lane == 0) {
       const uint32_t sK0 = smem_u32(sK), sV0 = smem_u32(sV), sQ0 = smem_u32(sQ);
       const uint32_t sDO0 = smem_u32(sDO), sX0 = smem_u32(sX);
-      auto issue_s = [&](int t) -> bool {  // S^T_t = K_j Q_t^T
+      auto issue_s = [&](int t) -> bool {  // S^T_t = K_j Q_t^T into S^T's columns
         const int st = t % C::kStages;
         if (!mbar_wait(&q_full[st], (t / C::kStages) & 1, abort_flag)) return false;
         if (t > 0 && !mbar_wait(s_free, (t - 1) & 1, abort_flag)) return false;
+        // d = 128: the columns held dQ_t-2 after S^T_t-1; it must have been read out
+        if (C::kDqT && t > 1 && !mbar_wait(dq_free, (t - 2) & 1, abort_flag)) return false;
         tc_fence_after();
         issue_qk<HD>(tmem + C::kColS, sK0, sQ0 + st * C::kTileBytes);
         umma_commit(s_full);
         return true;
       };
-      auto issue_dp = [&](int t) -> bool {  // dP^T_t = V_j dO_t^T
-        const int st = t % C::kStages;
-        if (!mbar_wait(&do_full[st], (t / C::kStages) & 1, abort_flag)) return false;
-        // at d = 128 these columns held dQ_t-1: it must have been read out
-        if (C::kDqOnDp && t > 0 && !mbar_wait(dq_free, (t - 1) & 1, abort_flag)) return false;
+      auto issue_dp = [&](int t) -> bool {  // dP^T_t = V_j dO_t^T (dS^T_t-1 already formed)
+        const int sd = t % C::kDoStages;
+        if (!mbar_wait(&do_full[sd], (t / C::kDoStages) & 1, abort_flag)) return false;
         tc_fence_after();
-        issue_qk<HD>(tmem + C::kColDP, sV0, sDO0 + st * C::kTileBytes);
+        issue_qk<HD>(tmem + C::kColDP, sV0, sDO0 + sd * C::kTileBytes);
         umma_commit(dp_full);
         return true;
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag) && issue_s(0) && issue_dp(0);
       for (int t = 0; ok && t < n; ++t) {
-        const int st = t % C::kStages;
-        if (t + 1 < n && !issue_s(t + 1)) { ok = false; break; }
+        const int st = t % C::kStages, sd = t % C::kDoStages;
         if (!mbar_wait(p_full, t & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        issue_x_kmajor<HD>(tmem + C::kColDV, sX0, sDO0 + st * C::kTileBytes, C::kIdescKV, t > 0);
+        issue_x_kmajor<HD>(tmem + C::kColDV, sX0, sDO0 + sd * C::kTileBytes, C::kIdescKV, t > 0);
         umma_commit(dv_done);
-        umma_commit(&do_empty[st]);
+        umma_commit(&do_empty[sd]);
+        if (t + 1 < n && !issue_s(t + 1)) { ok = false; break; }
         if (!mbar_wait(ds_full, t & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         issue_x_kmajor<HD>(tmem + C::kColDK, sX0, sQ0 + st * C::kTileBytes, C::kIdescKV, t > 0);
         umma_commit(&q_empty[st]);
-        if (!C::kDqOnDp && t > 0 && !mbar_wait(dq_free, (t - 1) & 1, abort_flag)) { ok = false; break; }
+        // dQ_t-1 must have been read out of the dQ columns
+        if (t > 0 && !mbar_wait(dq_free, (t - 1) & 1, abort_flag)) { ok = false; break; }
+        if constexpr (C::kDqT) {
+          // dQ^T_t goes where S^T_t+1 sits: wait until the compute warps have copied it out
+          const int last_s = t + 1 < n ? t + 1 : t;
+          if (!mbar_wait(s_free, last_s & 1, abort_flag)) { ok = false; break; }
+        }
         tc_fence_after();
         issue_dq<HD>(tmem + C::kColDQ, sX0, sK0);
         umma_commit(dq_full);
-        umma_commit(x_free);
         if (t + 1 < n && !issue_dp(t + 1)) { ok = false; break; }
       }
       // every MMA issued by this thread completes before TMEM is released
@@ -300,17 +404,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       volatile int never = 0;
       mbar_wait(drain, 0, &never);
     }
-  } else if (warp < 4) {
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------------ dQ read-out
+    const int w4 = warp % 4;
+    const uint32_t tQ = tmem + (static_cast<uint32_t>(w4 * 32) << 16) + C::kColDQ;
+    uint8_t *slot = sStage + w4 * C::kStageSlotBytes;
+    const int row_head = bh * p.Np;  // the head's first row in the accumulator's [BH * Np, d] view
+    for (int t = 0; t < n; ++t) {
+      const int i = qblock(t);
+      if (!__all_sync(0xffffffffu, mbar_wait(dq_full, t & 1, abort_flag))) break;
+      tc_fence_after();
+      read_out_dq<HD>(tQ, w4, lane, slot, &tm_dq, row_head + i * kBM, dq_free);
+    }
+    if (lane == 0) bulk_wait_group_all();  // every reduction has landed before the CTA retires
+    __syncwarp();
+  } else {
     // ------------------------------------------------------------------ compute: P^T, dS^T
-    const int r = threadIdx.x;  // key row within the block == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::kColS, tDP = tmem + lane_off + C::kColDP;
-    const float sl2 = p.scale_log2;
+    const int h = warp / 4;                   // query columns [64 h, 64 h + 64)
+    const int w4 = warp % 4;
+    const int r = threadIdx.x % 128;          // key row within the block == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(w4 * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS + 64 * h;
+    const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * h;
+    const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
     const bool key_live = jb * kBN + r < p.N;  // keys past N (zero-filled rows) get P = 0
+    const bool ragged_keys = (jb + 1) * kBN > p.N;
     bool ok = true;
     for (int t = 0; t < n; ++t) {
-      const int i = i_lo + t, st = t % C::kStages;
-      const float *vlse = sVec + st * C::kVecFloats, *vd = vlse + kBM;
+      const int i = qblock(t), st = t % C::kStages;
+      const float *vlse = sVec + st * C::kVecFloats + 64 * h, *vd = vlse + kBM;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, t & 1, abort_flag))) { ok = false; break; }
       // S^T_t was computed from this stage, so it has landed; waiting makes its LSE2 / D rows
       // visible to these threads
@@ -319,100 +441,94 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         break;
       }
       tc_fence_after();
-      float s[kBN];
-      tmem_ld32(tS + 0, reinterpret_cast<uint32_t *>(s));
+      float s[64];
+      tmem_ld32(tS, reinterpret_cast<uint32_t *>(s));
       tmem_ld32(tS + 32, reinterpret_cast<uint32_t *>(s) + 32);
-      tmem_ld32(tS + 64, reinterpret_cast<uint32_t *>(s) + 64);
-      tmem_ld32(tS + 96, reinterpret_cast<uint32_t *>(s) + 96);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
-      // P^T row: p_c = 2^(s_c scale log2(e) - LSE2_c); on the diagonal block (causal) key r is
-      // visible to query c only if r <= c
-      const bool diag = p.causal && i == jb;
-      uint32_t pk[kBN / 2];
+      // P^T: p = 2^(s scale log2(e) - LSE2_q); on the diagonal block (causal) key r is visible to
+      // query q only if r <= q, and keys past N are dropped
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        float p0 = ex2(fmaf(s[c], sl2, -vlse[c]));
-        float p1 = ex2(fmaf(s[c + 1], sl2, -vlse[c + 1]));
-        if (!key_live || (diag && c < r)) p0 = 0.f;
-        if (!key_live || (diag && c + 1 < r)) p1 = 0.f;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+      for (int c = 0; c < 64; c += 4) {
+        const float4 l4 = *reinterpret_cast<const float4 *>(vlse + c);
+        const uint64_t x01 = f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, f2_pack(-l4.x, -l4.y));
+        const uint64_t x23 = f2_fma(f2_pack(s[c + 2], s[c + 3]), sl2x2, f2_pack(-l4.z, -l4.w));
+        float x0, x1, x2, x3;
+        f2_unpack(x01, x0, x1);
+        f2_unpack(x23, x2, x3);
+        s[c] = ex2(x0);
+        s[c + 1] = ex2(x1);
+        s[c + 2] = ex2(x2);
+        s[c + 3] = ex2(x3);
       }
-      if (t > 0 && !__all_sync(0xffffffffu, mbar_wait(x_free, (t - 1) & 1, abort_flag))) {
-        ok = false;
-        break;
+      if ((p.causal && i == jb) || ragged_keys) {
+        const int qmin = r - 64 * h;  // visible iff local column >= qmin (diagonal block)
+        const bool diag = p.causal && i == jb;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (!key_live || (diag && c < qmin)) s[c] = 0.f;
       }
-      store_p_row(sX, r, pk);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
+      if (t > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (t - 1) & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+      }
+      store_x_half(sX, r, h, pk);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      // dS^T row: ds_c = p_c (dP_c - D_c), with the bf16 p the tensor core used for dV
+      // dS^T: ds = p (dP - D_q), with the bf16 p the tensor core used for dV
       if (!__all_sync(0xffffffffu, mbar_wait(dp_full, t & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      uint32_t dk[kBN / 2];
+      uint32_t dk[32];
 #pragma unroll
-      for (int cc = 0; cc < kBN; cc += 32) {
+      for (int cc = 0; cc < 64; cc += 32) {
         uint32_t dp[32];
         tmem_ld32(tDP + cc, dp);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const uint32_t pp = pk[(cc + e) / 2];
-          const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
-          const float d0 = p0 * (__uint_as_float(dp[e]) - vd[cc + e]);
-          const float d1 = p1 * (__uint_as_float(dp[e + 1]) - vd[cc + e + 1]);
-          dk[(cc + e) / 2] = pack_bf16x2(d0, d1);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 d4 = *reinterpret_cast<const float4 *>(vd + cc + e);
+          const uint32_t pa = pk[(cc + e) / 2], pb = pk[(cc + e) / 2 + 1];
+          const uint64_t g01 = f2_mul(f2_pack(__uint_as_float(pa << 16), __uint_as_float(pa & 0xffff0000u)),
+                                      f2_sub(f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                             f2_pack(d4.x, d4.y)));
+          const uint64_t g23 = f2_mul(f2_pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xffff0000u)),
+                                      f2_sub(f2_pack(__uint_as_float(dp[e + 2]), __uint_as_float(dp[e + 3])),
+                                             f2_pack(d4.z, d4.w)));
+          float a0, a1, a2, a3;
+          f2_unpack(g01, a0, a1);
+          f2_unpack(g23, a2, a3);
+          dk[(cc + e) / 2] = pack_bf16x2(a0, a1);
+          dk[(cc + e) / 2 + 1] = pack_bf16x2(a2, a3);
         }
       }
       tc_fence_before();
       if (!__all_sync(0xffffffffu, mbar_wait(dv_done, t & 1, abort_flag))) { ok = false; break; }
-      store_p_row(sX, r, dk);
+      store_x_half(sX, r, h, dk);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
     }
-    // epilogue: dV_j and dK_j (times scale) once every MMA of the loop has completed
-    if (ok && __all_sync(0xffffffffu, mbar_wait(x_free, (n - 1) & 1, abort_flag))) {
+    // dV_j and dK_j (times scale) once every MMA has completed
+    if (ok && __all_sync(0xffffffffu, mbar_wait(dq_full, (n - 1) & 1, abort_flag))) {
       tc_fence_after();
       const size_t grow = static_cast<size_t>(bh) * p.N + jb * kBN + r;
-      store_grad_row<HD>(tmem + lane_off + C::kColDV, 1.f, p.dv, p.g_f32, grow, key_live);
-      store_grad_row<HD>(tmem + lane_off + C::kColDK, p.scale, p.dk, p.g_f32, grow, key_live);
-    }
-  } else {
-    // ------------------------------------------------------------------ dQ read-out
-    const int qr = threadIdx.x - 128;  // query row within the block == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
-    const uint32_t tQ = tmem + lane_off + C::kColDQ;
-    for (int t = 0; t < n; ++t) {
-      const int row = (i_lo + t) * kBM + qr;
-      if (!__all_sync(0xffffffffu, mbar_wait(dq_full, t & 1, abort_flag))) break;
-      tc_fence_after();
-      float *dst = p.dq_acc + (static_cast<size_t>(bh) * p.Np + row) * HD;
-#pragma unroll
-      for (int cc = 0; cc < HD; cc += 32) {
-        uint32_t v[32];
-        tmem_ld32(tQ + cc, v);
-        tmem_wait_ld();
-        if (row < p.N) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            atomicAdd(reinterpret_cast<float4 *>(dst + cc + 4 * e),
-                      make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                  __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
+      store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDV, h * (HD / 2), 1.f, p.dv, p.g_f32,
+                                   grow, key_live);
+      store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDK, h * (HD / 2), p.scale, p.dk,
+                                   p.g_f32, grow, key_live);
     }
   }
 
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(*tmem_slot, C::kTmemCols);
   }

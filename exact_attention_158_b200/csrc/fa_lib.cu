@@ -107,6 +107,21 @@ bool encode_bhnd(CUtensorMap *map, const void *base, int d, int N, int BH) {
   return r == CUDA_SUCCESS;
 }
 
+// The backward's fp32 dQ accumulator [rows, d] as a 2-D tensor for bulk reductions: boxes of
+// 32 features (128 bytes) x box_rows rows, 128-byte swizzle.
+bool encode_dq_acc(CUtensorMap *map, float *base, int d, long long rows, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 4};
+  cuuint32_t box[2] = {32, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
@@ -240,9 +255,14 @@ fa_status launch_bwd(DeviceInfo &dev, const void *q, const void *k, const void *
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
+  CUtensorMap tdq;
+  if (!encode_dq_acc(&tdq, dq_acc, HD, static_cast<long long>(prow), C::kBoxRows)) {
+    t_last_error = "cuTensorMapEncodeTiled failed";
+    return FA_ERR_LAUNCH;
+  }
   const long long units = static_cast<long long>(BH) * p.nkb;
   fa::fa_bwd_kernel<HD><<<static_cast<unsigned>(units), fa::kBwdThreads, C::kSmemBytes, stream>>>(
-      tq, tk, tv, tdo, p);
+      tq, tk, tv, tdo, tdq, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return launch_failed(e);
   const long long post_threads = static_cast<long long>(BH) * N * kRowThreads;
   fa::fa_bwd_dq_kernel<HD><<<static_cast<unsigned>((post_threads + 255) / 256), 256, 0, stream>>>(
