@@ -34,6 +34,13 @@
  * cache, exact attention for the compute), so query t of the chunk sits at position L - Lq + t and,
  * when causal, sees keys 0 .. L - Lq + t; otherwise all L keys.
  *
+ * oracle_tree_attention is the verification step of speculative decoding ("LLM study notes",
+ * speculative decoding: the draft model proposes candidate tokens arranged as a tree, and the target
+ * model scores every node of the tree in one forward pass with tree attention).  The tree's T
+ * nodes are the last T of the sequence's L cached tokens; node t sees the L - T context tokens and
+ * the nodes u whose bit u is set in mask[t] (its ancestors and itself, for a tree).  A row that
+ * sees no key at all has O = 0 and LSE = -inf.
+ *
  * oracle_attention_bwd is the backward pass: the gradients of the scalar sum_i dO[i] . O[i] with
  * respect to Q, K and V for a given dO.  The pages describe the backward only in prose ("Paged vs
  * Flash attention", training: gradients from the stored intermediate results, block by block;
@@ -513,6 +520,87 @@ int oracle_attention_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
                      nheads * t / nthreads, nheads * (t + 1) / nthreads};
         jobs[t] = j;
         pthread_create(&th[t], NULL, bwd_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+    free(jobs);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* tree attention: T draft nodes per sequence, visibility of the tree part given by bit masks  */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *q, *kp, *vp;
+    const int32_t *table, *lens;
+    const uint64_t *mask;
+    int max_blocks, H, T, d, page;
+    double scale;
+    double *o, *lse;
+    int64_t first, last; /* range of (s, h, t) rows */
+} tree_job;
+
+static void *tree_worker(void *arg)
+{
+    tree_job *jb = (tree_job *)arg;
+    const int H = jb->H, d = jb->d, page = jb->page, T = jb->T;
+    int64_t maxlen = (int64_t)jb->max_blocks * page;
+    double *s = (double *)malloc(sizeof(double) * (size_t)maxlen);
+    const uint16_t **kr = (const uint16_t **)malloc(sizeof(void *) * (size_t)maxlen);
+    const uint16_t **vr = (const uint16_t **)malloc(sizeof(void *) * (size_t)maxlen);
+    for (int64_t r = jb->first; r < jb->last; ++r) {
+        int64_t t = r % T, u = r / T, sq = u / H, h = u % H;
+        int64_t L = jb->lens[sq], ctx = L - T;
+        uint64_t m = jb->mask[sq * T + t];
+        int64_t n_keys = 0;
+        for (int64_t key = 0; key < L; ++key) {
+            if (key >= ctx && !((m >> (key - ctx)) & 1u))
+                continue; /* a tree node this one does not see */
+            int64_t blk = jb->table[sq * jb->max_blocks + key / page];
+            int64_t off = ((blk * H + h) * page + key % page) * d;
+            kr[n_keys] = jb->kp + off;
+            vr[n_keys] = jb->vp + off;
+            ++n_keys;
+        }
+        if (n_keys == 0) {
+            for (int c = 0; c < d; ++c)
+                jb->o[r * d + c] = 0.0;
+            jb->lse[r] = -INFINITY;
+            continue;
+        }
+        const uint16_t *node_q = jb->q + r * d;
+        attend_row(node_q, kr, vr, n_keys, d, jb->scale, s, jb->o + r * d, jb->lse + r);
+    }
+    free(s);
+    free(kr);
+    free(vr);
+    return NULL;
+}
+
+/* q [S,H,T,d]; pools [num_blocks,H,page,d]; table [S,max_blocks]; lens [S] (each >= T);
+ * mask [S,T] (bit u of mask[s*T+t]: node t sees node u; T <= 64); o [S,H,T,d]; lse [S,H,T]. */
+int oracle_tree_attention(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool,
+                          const int32_t *block_table, int max_blocks, const int32_t *seq_lens,
+                          const uint64_t *mask, int S, int H, int T, int d, int page, double scale,
+                          double *o, double *lse, int nthreads)
+{
+    if (S < 1 || H < 1 || T < 1 || T > 64 || d < 1 || page < 1 || max_blocks < 1 || nthreads < 1)
+        return 1;
+    for (int s = 0; s < S; ++s)
+        if (seq_lens[s] < T || seq_lens[s] > (int64_t)max_blocks * page)
+            return 1;
+    int64_t rows = (int64_t)S * H * T;
+    if (nthreads > rows)
+        nthreads = (int)rows;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    tree_job *jobs = (tree_job *)malloc(sizeof(tree_job) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) {
+        tree_job j = {q, k_pool, v_pool, block_table, seq_lens, mask, max_blocks, H, T, d, page,
+                      scale, o, lse, rows * t / nthreads, rows * (t + 1) / nthreads};
+        jobs[t] = j;
+        pthread_create(&th[t], NULL, tree_worker, &jobs[t]);
     }
     for (int t = 0; t < nthreads; ++t)
         pthread_join(th[t], NULL);

@@ -24,6 +24,7 @@ _lib = None
 _u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
 _i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+_u64p = np.ctypeslib.ndpointer(dtype=np.uint64, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 _i64 = ctypes.c_int64
 _int = ctypes.c_int
@@ -54,6 +55,10 @@ class OracleLib:
                                             _int, _int, _dbl, _f64p, _f64p, _int]
         lib.oracle_prefill_paged.argtypes = [_u16p, _u16p, _u16p, _i32p, _int, _i32p, _int, _int,
                                              _int, _int, _int, _int, _dbl, _f64p, _f64p, _int]
+        lib.oracle_tree_attention.argtypes = [_u16p, _u16p, _u16p, _i32p, _int, _i32p, _u64p,
+                                              _int, _int, _int, _int, _int, _dbl, _f64p, _f64p,
+                                              _int]
+        lib.oracle_tree_attention.restype = ctypes.c_int
         lib.oracle_attention_bwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _i64, _int, _int, _dbl,
                                              _i64p, _i64, _f64p, _f64p, _f64p, _int]
         for f in (lib.oracle_attention, lib.oracle_attention_rows, lib.oracle_attention_probs,
@@ -110,6 +115,25 @@ class OracleLib:
         if rc:
             raise ValueError("oracle_flash_alg1: bad arguments")
         return O, l, m
+
+    def tree_attention(self, q, k_pool, v_pool, block_table, seq_lens, tree_mask, scale: float,
+                       page: int = 16, nthreads: int | None = None):
+        """Tree verification.  q [S,H,T,d] are the tree's nodes, the last T of each sequence's
+        cached tokens; tree_mask [S,T] (uint64 bit patterns, any integer dtype): bit u of entry t
+        set when node t sees node u.  Returns (o [S,H,T,d], lse [S,H,T])."""
+        q, k_pool, v_pool = _bits(q), _bits(k_pool), _bits(v_pool)
+        table = np.ascontiguousarray(block_table, dtype=np.int32)
+        lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        mask = np.ascontiguousarray(np.asarray(tree_mask).astype(np.int64).view(np.uint64))
+        S, H, T, d = q.shape
+        o = np.empty((S, H, T, d), np.float64)
+        lse = np.empty((S, H, T), np.float64)
+        rc = self.lib.oracle_tree_attention(q, k_pool, v_pool, table, table.shape[1], lens, mask,
+                                            S, H, T, d, page, scale, o, lse,
+                                            nthreads or default_threads())
+        if rc:
+            raise ValueError("oracle_tree_attention: bad arguments")
+        return o, lse
 
     def attention_bwd(self, q, k, v, dout, causal: bool, scale: float, heads=None,
                       nthreads: int | None = None):
@@ -214,3 +238,7 @@ def prefill_paged(*a, **kw):
 
 def attention_bwd(*a, **kw):
     return default().attention_bwd(*a, **kw)
+
+
+def tree_attention(*a, **kw):
+    return default().tree_attention(*a, **kw)

@@ -15,6 +15,8 @@ The facts used:
   block sizes give the plain result;
 * a paged KV cache is only a relocation of logically contiguous rows ("LLM study notes", paged
   attention);
+* a draft-token tree is verified in one pass, each node continuing the context along its path
+  ("LLM study notes", speculative decoding), so a node sees its ancestors and itself;
 * the backward pass returns the gradients of sum(dO * O) with respect to Q, K and V (the pages
   describe it in prose only: "Paged vs Flash attention", training; "Flash Attention" (myungum),
   section 1, recomputation), so it must agree with central finite differences of the forward
@@ -392,7 +394,66 @@ def pin_bwd_closed_forms(orc):
             close(x, y, 1e-11, f"key shift leaves {name} unchanged causal={causal}")
 
 
+def _ancestors_or_self(parents, t):
+    seen = set()
+    while t >= 0:
+        seen.add(t)
+        t = parents[t]
+    return seen
+
+
+def pin_tree_attention(orc):
+    """Tree verification: node t of a draft tree continues the context along the path root..t, so
+    it sees the L - T context tokens and exactly its ancestors and itself among the tree's nodes
+    (walked here from the parent lists, not from the masks).  scipy softmax/logsumexp over the
+    gathered rows; a chain tree is the causal chunk of the same T tokens; with no context a star
+    tree gives each node its own value row; a node that sees nothing gets O = 0, LSE = -inf."""
+    case = W.DecodeCase("pintree", S=3, H=2, d=16, lens=[20, 41, 64])
+    for shape in ("random", "star", "chain"):
+        inp = W.make_tree_verify(case, 12, shape)
+        q = W.bf16_bits(inp["q"])
+        kp, vp = W.bf16_bits(inp["k_pool"]), W.bf16_bits(inp["v_pool"])
+        table, lens = inp["block_table"].numpy(), inp["seq_lens"].numpy()
+        o, lse = orc.tree_attention(q, kp, vp, table, lens, inp["tree_mask"].numpy(), case.scale)
+        for s, L in enumerate(case.lens):
+            ctx = L - 12
+            for h in range(case.H):
+                Kc, Vc = _gather(kp, vp, table, s, h, L)
+                S_ = case.scale * widen(q[s, h]) @ widen(Kc).T
+                for t in range(12):
+                    vis = _ancestors_or_self(inp["parents"][s], t)
+                    for u in range(12):
+                        if u not in vis:
+                            S_[t, ctx + u] = -np.inf
+                close(o[s, h], sps.softmax(S_, axis=1) @ widen(Vc), 1e-13,
+                      f"tree {shape} O s={s} h={h}")
+                close(lse[s, h], sps.logsumexp(S_, axis=1), 1e-13, f"tree {shape} LSE s={s} h={h}")
+        if shape == "chain":
+            oc, lc = orc.prefill_paged(q, kp, vp, table, lens, True, case.scale)
+            close(o, oc, 0.0, "chain tree vs causal chunk")
+            close(lse, lc, 0.0, "chain tree vs causal chunk LSE")
+    # no context: a star tree leaves each node only itself
+    case0 = W.DecodeCase("pintree0", S=1, H=2, d=16, lens=[9])
+    inp = W.make_tree_verify(case0, 9, "star")
+    q = W.bf16_bits(inp["q"])
+    kp, vp = W.bf16_bits(inp["k_pool"]), W.bf16_bits(inp["v_pool"])
+    table, lens = inp["block_table"].numpy(), inp["seq_lens"].numpy()
+    o, lse = orc.tree_attention(q, kp, vp, table, lens, inp["tree_mask"].numpy(), case0.scale)
+    for h in range(2):
+        Kc, Vc = _gather(kp, vp, table, 0, h, 9)
+        close(o[0, h], widen(Vc), 0.0, "star without context: O = own V")
+        close(lse[0, h], case0.scale * np.sum(widen(q[0, h]) * widen(Kc), axis=1), 1e-13,
+              "star without context: LSE = own score")
+    # a node that sees nothing
+    mask = inp["tree_mask"].numpy().copy()
+    mask[0, 4] = 0
+    o, lse = orc.tree_attention(q, kp, vp, table, lens, mask, case0.scale)
+    close(o[0, :, 4], np.zeros((2, 16)), 0.0, "empty row: O = 0")
+    assert np.all(np.isneginf(lse[0, :, 4])), "empty row: LSE = -inf"
+
+
 ALL_PINS = [pin_uniform_scores, pin_single_key, pin_dominant_score, pin_two_keys_logistic,
             pin_shift_invariance, pin_rows_sum_to_one, pin_library_softmax, pin_permutation,
             pin_linear_in_v, pin_tiled_algorithm, pin_paged_decode, pin_paged_prefill,
-            pin_bwd_finite_differences, pin_bwd_autograd, pin_bwd_closed_forms]
+            pin_bwd_finite_differences, pin_bwd_autograd, pin_bwd_closed_forms,
+            pin_tree_attention]

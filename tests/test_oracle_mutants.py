@@ -50,6 +50,10 @@ MUTANTS = {
     "bwd_causal_ignored": ("const int64_t n_keys = causal ? i + 1 : N; /* the keys row i sees */",
                            "const int64_t n_keys = N;"),
     "bwd_row_not_normalised": ("            p[j] /= l;\n        /* dP row", "            p[j] /= 1.0;\n        /* dP row"),
+    "tree_mask_ignored": ("if (key >= ctx && !((m >> (key - ctx)) & 1u))", "if (0)"),
+    "tree_offset": ("int64_t L = jb->lens[sq], ctx = L - T;", "int64_t L = jb->lens[sq], ctx = L - T + 1;"),
+    "tree_bit_order": ("if (key >= ctx && !((m >> (key - ctx)) & 1u))",
+                       "if (key >= ctx && !((m >> (T - 1 - (key - ctx))) & 1u))"),
 }
 
 

@@ -1,3 +1,4 @@
+import pytest
 """The seeded input generator and the workload shapes (no GPU)."""
 import json
 import math
@@ -97,3 +98,17 @@ def test_paged_prefill_flops_counts_visible_pairs():
         pairs = sum(1 for L in lens for t in range(Lq) for key in range(L)
                     if not causal or key <= L - Lq + t)
         assert W.paged_prefill_flops(lens, H, d, Lq, causal) == 4 * d * H * pairs
+
+
+def test_tree_visibility_is_the_ancestor_set():
+    for shape in ("random", "star", "chain"):
+        for parents in W.random_tree_parents(5, 3, 40, shape):
+            bits = W.tree_visibility(parents)
+            for t in range(40):
+                anc, u = set(), t
+                while u >= 0:
+                    anc.add(u)
+                    u = parents[u]
+                assert {u for u in range(40) if bits[t] >> u & 1} == anc
+    with pytest.raises(ValueError):
+        W.tree_visibility([0])

@@ -30,7 +30,7 @@ from dataclasses import dataclass, field
 import torch
 
 BASE_SEED = 158
-TID_Q, TID_K, TID_V, TID_LENS, TID_PERM, TID_PEAKS, TID_DO = 1, 2, 3, 4, 5, 6, 7
+TID_Q, TID_K, TID_V, TID_LENS, TID_PERM, TID_PEAKS, TID_DO, TID_TREE = 1, 2, 3, 4, 5, 6, 7, 8
 PAGE_SIZE = 16
 
 _M64 = (1 << 64) - 1
@@ -279,6 +279,59 @@ def paged_prefill_flops(lens, H: int, d: int, Lq: int, causal: bool) -> int:
     pairs = 0
     for L in lens:
         pairs += Lq * (L - Lq) + Lq * (Lq + 1) // 2 if causal else Lq * L
+    return 4 * d * H * pairs
+
+
+def random_tree_parents(seed: int, S: int, T: int, shape: str = "random") -> list[list[int]]:
+    """Draft-token trees, one per sequence, as parent lists in topological order: node t's parent
+    is -1 (it follows the context directly) or an earlier node.  shape: "random" (parent of t
+    uniform over -1 .. t-1, seeded), "chain" (t - 1), "star" (all -1)."""
+    trees = []
+    for s in range(S):
+        if shape == "chain":
+            trees.append([t - 1 for t in range(T)])
+        elif shape == "star":
+            trees.append([-1] * T)
+        else:
+            draws = uniform_ints(seed, TID_TREE, T, 0, 1 << 30, start=s * T)
+            trees.append([(w % (t + 1)) - 1 for t, w in enumerate(draws)])
+    return trees
+
+
+def tree_visibility(parents: list[int]) -> list[int]:
+    """Bit u of entry t is set when node u is node t itself or one of its ancestors: the draft
+    tokens on the path from the context to t (the sequence node t continues)."""
+    bits = []
+    for t, par in enumerate(parents):
+        if not -1 <= par < t:
+            raise ValueError("parents must point to an earlier node or -1")
+        bits.append((1 << t) | (bits[par] if par >= 0 else 0))
+    return bits
+
+
+def make_tree_verify(case: "DecodeCase", T: int, shape: str = "random", device="cpu"):
+    """Tree verification over a paged cache: the decode case's pool, table and lengths (each length
+    >= T, the last T cached tokens being the tree's nodes in topological order), q [S,H,T,d] for the
+    nodes, and the visibility masks as int64 [S, T] (the bit pattern of uint64; T <= 64)."""
+    if not 1 <= T <= 64:
+        raise ValueError("tree size must be in [1, 64]")
+    inp = make_paged_prefill(case, T, device)
+    parents = random_tree_parents(case.seed, case.S, T, shape)
+    masks = [tree_visibility(p) for p in parents]
+    signed = [[m - (1 << 64) if m >= 1 << 63 else m for m in row] for row in masks]
+    inp["parents"] = parents
+    inp["tree_mask"] = torch.tensor(signed, dtype=torch.int64).to(device)
+    inp["T"] = T
+    return inp
+
+
+def tree_verify_flops(lens, masks, H: int, d: int) -> int:
+    """Matmul FLOPs of tree verification: 4 d per visible (node, key) pair; node t of a length-L
+    context sees the L - T context tokens and the nodes set in its mask."""
+    pairs = 0
+    for L, row in zip(lens, masks):
+        T = len(row)
+        pairs += sum((L - T) + bin(m & ((1 << 64) - 1)).count("1") for m in row)
     return 4 * d * H * pairs
 
 
