@@ -15,8 +15,8 @@ Extra keys: `roofline` (prefill kernel vs the measured dense bf16 peak), `cpu_ba
 oracle on this host's cores, a bounded row sample), `e2e` (the same metric through the Python API
 with Q/K/V copied from pinned host memory and O/LSE copied back inside the timed region), `sweep`
 (the sequence-length grid, d = 128 and d = 64), `decode` (paged decode GB/s vs HBM),
-`paged_prefill` (chunked prefill through the block table, TFLOP/s), `backward` (fa_bwd TFLOP/s)
-and `clocks`.
+`paged_prefill` (chunked prefill through the block table, TFLOP/s), `backward` (fa_bwd TFLOP/s),
+`tree` (draft-tree verification TFLOP/s) and `clocks`.
 """
 from __future__ import annotations
 
@@ -286,6 +286,40 @@ def bench_paged_prefill(fa, args, dev, flush, stream, pk):
             "launches_per_step": 1}
 
 
+def bench_tree(fa, args, dev, flush, stream, pk):
+    """Draft-tree verification: 32 sequences, 64-node seeded random trees after contexts of
+    U[2048, 8192] tokens, H32 d128, one fa_tree_attention launch per step."""
+    T = 64
+    case = W.DecodeCase("tree_verify", S=32, H=32, d=128, len_lo=2048 + T, len_hi=8192 + T)
+    inp = W.make_tree_verify(case, T, "random", device=dev)
+    o = torch.empty_like(inp["q"])
+    lse = torch.empty(inp["q"].shape[:3], dtype=torch.float32, device=dev)
+    fn = lambda: fa.fa_tree_attention(inp["q"], inp["k_pool"], inp["v_pool"], inp["block_table"],
+                                      inp["seq_lens"], inp["tree_mask"], scale=case.scale, out=o,
+                                      lse=lse)
+    torch.cuda.nvtx.range_push("bench_tree_timed")
+    ts = time_launches(fn, args.sweep_steps, 3, flush, stream)
+    torch.cuda.nvtx.range_pop()
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during the tree bench")
+    ms = statistics.median(ts)
+    masks = [W.tree_visibility(p) for p in inp["parents"]]
+    flops = W.tree_verify_flops(inp["lens"], masks, case.H, case.d)
+    nbytes = W.tree_verify_bytes(inp["lens"], case.H, case.d, T)
+    tf = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    # 64 queries per (sequence, head) against every cached key: about 64 FLOP per byte of K/V,
+    # below the ridge point (measured peak FLOP/s over measured bandwidth), so HBM bounds it
+    return {"metric": "draft-tree verification over a paged cache, TFLOP/s",
+            "workload": "32 seqs, 64-node random draft trees, context U[2048,8192], H32 d128, "
+            "16-token pages, permuted block table",
+            "ms": round(ms, 4), "value": round(tf, 2), "unit": "TFLOP/s",
+            "algorithmic_bytes": nbytes, "flop_per_byte": round(flops / nbytes, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4)},
+            "launches_per_step": 1}
+
+
 def bench_backward(fa, args, dev, flush, stream, pk):
     """fa_bwd on the headline shape (B8 H16 N2048 d128), non-causal and causal.  FLOPs are the five
     matmuls per (query, key) pair: 2.5x the forward's 4 B H N^2 d (halved causal)."""
@@ -326,6 +360,8 @@ def bench_ours(args, rank, world):
     pk = peaks()
     if args.only == "decode":
         return {"metric": METRIC, "decode": bench_decode(fa, args, dev, flush, stream, pk)}
+    if args.only == "tree":
+        return {"metric": METRIC, "tree": bench_tree(fa, args, dev, flush, stream, pk)}
     if args.only == "backward":
         return {"metric": METRIC, "backward": bench_backward(fa, args, dev, flush, stream, pk)}
     if args.only == "paged":
@@ -452,8 +488,11 @@ def bench_ours(args, rank, world):
     # ---- backward (tensor bound)
     bwd = None if args.no_backward else bench_backward(fa, args, dev, flush, stream, pk)
 
+    # ---- draft-tree verification (tensor bound, short query tiles)
+    tree = None if args.no_tree else bench_tree(fa, args, dev, flush, stream, pk)
+
     result.update({"e2e": e2e, "sweep": sweep, "decode": dec, "paged_prefill": paged,
-                   "backward": bwd})
+                   "backward": bwd, "tree": tree})
     return result
 
 
@@ -488,10 +527,11 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-paged", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-tree", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="sequences in the decode workload (64 is the benchmark; fewer for profiling)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "paged", "backward"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "paged", "backward", "tree"],
                     default="all",
                     help="prefill: the headline loop alone; decode / paged: the paged decode or "
                     "chunked prefill loop alone")

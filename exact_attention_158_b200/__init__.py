@@ -18,6 +18,7 @@ import torch
 from . import build as _build
 
 __all__ = ["fa_fwd", "fa_bwd", "fa_decode_paged", "fa_decode_paged_noalloc", "fa_prefill_paged",
+           "fa_tree_attention",
            "fa_decode_workspace_size",
            "NOALLOC_SCRATCH_BYTES", "device_status",
            "FaError", "library_path", "load_library", "EXPORTED_SYMBOLS", "STATUS"]
@@ -27,7 +28,8 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 FA_OUT_BF16, FA_OUT_F32 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
-                    "fa_decode_paged_noalloc", "fa_prefill_paged", "fa_bwd_workspace_size",
+                    "fa_decode_paged_noalloc", "fa_prefill_paged", "fa_tree_attention",
+                    "fa_bwd_workspace_size",
                     "fa_bwd", "fa_get_device_status",
                     "fa_status_string",
                     "fa_last_error_string", "fa_version", "fa_selftest_wait_timeout")
@@ -71,6 +73,9 @@ def load_library():
     lib.fa_prefill_paged.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, i32, vp, i32, i32, i32, i32,
                                      i32, f32, vp]
     lib.fa_prefill_paged.restype = i32
+    lib.fa_tree_attention.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, vp, i32, vp, i32, i32, i32,
+                                      i32, f32, vp]
+    lib.fa_tree_attention.restype = i32
     lib.fa_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
@@ -221,6 +226,43 @@ def fa_bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = No
                         _stream_handle(stream))
     _check(st, "fa_bwd")
     return dq, dk, dv
+
+
+def fa_tree_attention(q, k_pool, v_pool, block_table, seq_lens, tree_mask,
+                      scale: float | None = None, out_dtype=torch.bfloat16, out=None, lse=None,
+                      return_lse: bool = True, stream=None):
+    """Tree verification: q bf16 [S, H, T, d] holds the T draft nodes, the last T cached tokens of
+    each sequence; tree_mask int64 [S, T] (uint64 bit patterns: bit u of entry t set when node t
+    sees node u; T <= 64).  Pools, table and lengths as for fa_prefill_paged.
+    Returns (o [S, H, T, d], lse fp32 [S, H, T] or None)."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool")):
+        _require(t, n)
+    _require(block_table, "block_table", torch.int32)
+    _require(seq_lens, "seq_lens", torch.int32)
+    _require(tree_mask, "tree_mask", torch.int64)
+    S, H, T, d = q.shape
+    P = k_pool.shape[0]
+    if k_pool.shape != (P, H, 16, d) or v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool / v_pool must be [num_blocks, H, 16, d]")
+    if block_table.dim() != 2 or block_table.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_table must be [S, max_blocks] and seq_lens [S]")
+    if tree_mask.shape != (S, T):
+        raise ValueError("tree_mask must be [S, T]")
+    code = _out_code(out_dtype)
+    if out is None:
+        out = torch.empty((S, H, T, d), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((S, H, T), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib.fa_tree_attention(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                   block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(),
+                                   P, tree_mask.data_ptr(), out.data_ptr(), code,
+                                   lse.data_ptr() if lse is not None else None, S, H, T, d,
+                                   float(scale) if scale is not None else 0.0,
+                                   _stream_handle(stream))
+    _check(st, "fa_tree_attention")
+    return out, lse
 
 
 def fa_prefill_paged(q, k_pool, v_pool, block_table, seq_lens, causal: bool = True,

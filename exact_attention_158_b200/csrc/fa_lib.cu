@@ -528,11 +528,13 @@ fa_status fa_decode_paged_noalloc(const void *q, const void *k_pool, const void 
   return e == cudaSuccess ? FA_OK : launch_failed(e);
 }
 
-fa_status fa_prefill_paged(const void *q, const void *k_pool, const void *v_pool,
-                           const int32_t *block_table, int max_blocks_per_seq,
-                           const int32_t *seq_lens, int num_blocks, void *o, fa_out_dtype o_dtype,
-                           float *lse, int S, int H, int Lq, int d, int causal, float scale,
-                           fa_stream_t stream) {
+// Shared body of fa_prefill_paged and fa_tree_attention (tree_mask null: plain or causal chunk).
+static fa_status prefill_paged_impl(const void *q, const void *k_pool, const void *v_pool,
+                             const int32_t *block_table, int max_blocks_per_seq,
+                                    const int32_t *seq_lens, int num_blocks,
+                                    const uint64_t *tree_mask, void *o, fa_out_dtype o_dtype,
+                                    float *lse, int S, int H, int Lq, int d, int causal,
+                                    float scale, fa_stream_t stream) {
   if (!q || !k_pool || !v_pool || !block_table || !seq_lens || !o) return FA_ERR_INVALID_ARG;
   if (S < 1 || H < 1 || Lq < 1 || max_blocks_per_seq < 1 || num_blocks < 1) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
@@ -580,9 +582,37 @@ fa_status fa_prefill_paged(const void *q, const void *k_pool, const void *v_pool
   p.max_blocks = max_blocks_per_seq;
   p.num_blocks = num_blocks;
   p.H = H;
+  p.tree_mask = tree_mask;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128) return launch_prefill<128, true>(*dev, tq, tk, tv, p, s);
   return launch_prefill<64, true>(*dev, tq, tk, tv, p, s);
+}
+
+fa_status fa_prefill_paged(const void *q, const void *k_pool, const void *v_pool,
+                           const int32_t *block_table, int max_blocks_per_seq,
+                           const int32_t *seq_lens, int num_blocks, void *o, fa_out_dtype o_dtype,
+                           float *lse, int S, int H, int Lq, int d, int causal, float scale,
+                           fa_stream_t stream) {
+  return prefill_paged_impl(q, k_pool, v_pool, block_table, max_blocks_per_seq, seq_lens,
+                            num_blocks, nullptr, o, o_dtype, lse, S, H, Lq, d, causal, scale,
+                            stream);
+}
+
+fa_status fa_tree_attention(const void *q, const void *k_pool, const void *v_pool,
+                            const int32_t *block_table, int max_blocks_per_seq,
+                            const int32_t *seq_lens, int num_blocks, const uint64_t *tree_mask,
+                            void *o, fa_out_dtype o_dtype, float *lse, int S, int H, int T, int d,
+                            float scale, fa_stream_t stream) {
+  if (!tree_mask) return FA_ERR_INVALID_ARG;
+  if (T < 1 || T > 64) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(tree_mask) & 7u) return FA_ERR_ALIGNMENT;
+  if (S >= 1 && H >= 1 && (d == 64 || d == 128)) {
+    const size_t o_bytes =
+        static_cast<size_t>(S) * H * T * d * (o_dtype == FA_OUT_F32 ? 4 : 2);
+    if (overlaps(o, o_bytes, tree_mask, static_cast<size_t>(S) * T * 8)) return FA_ERR_INVALID_ARG;
+  }
+  return prefill_paged_impl(q, k_pool, v_pool, block_table, max_blocks_per_seq, seq_lens,
+                            num_blocks, tree_mask, o, o_dtype, lse, S, H, T, d, 0, scale, stream);
 }
 
 fa_status fa_get_device_status(fa_stream_t stream) {

@@ -80,6 +80,10 @@ struct PrefillParams {
   const int32_t *seq_lens;
   const int32_t *block_table;
   int max_blocks, num_blocks, H;
+  // tree verification (paged mode, causal = 0): the N queries are the nodes of a draft-token tree,
+  // the last N cached tokens in topological order; bit u of tree_mask[s * N + t] set when node t
+  // sees node u (N <= 64).  Null otherwise.
+  const uint64_t *tree_mask;
 };
 
 // Key count of unit (b, h) and the position of its first query among the keys.
@@ -593,6 +597,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int n = tile_blocks(p, kv, pr, wg);
       if (n == 0) continue;
       const int qrow = pr * 2 * kBM + wg * kBM + row;
+      const bool tree = kPaged && p.tree_mask != nullptr;
+      const uint64_t tmask =
+          (tree && qrow < p.N) ? p.tree_mask[static_cast<size_t>(w.bh / p.H) * p.N + qrow] : 0ull;
       float m_ref = -INFINITY, l = 0.f, lr = 0.f;
       for (int j = 0; j < n; ++j) {
         // the decision to go on must be warp-uniform: tcgen05.ld/st below are warp-collective
@@ -614,10 +621,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         bool edge;
         if constexpr (kPaged)
           edge = (p.causal && (j + 1) * kBN - 1 > kv.q_off + pr * 2 * kBM + wg * kBM) ||
-                 ((j + 1) * kBN > kv.L);
+                 ((j + 1) * kBN > kv.L) || (tree && (j + 1) * kBN > kv.q_off);
         else  // q_off = 0, L = N: only a causal tile's diagonal block and a ragged last block
           edge = (p.causal && j == n - 1) || ((j + 1) * kBN > p.N && (p.N % kBN) != 0);
-        if (edge) {
+        if (kPaged && tree && edge) {
+          // context keys (< q_off) are visible; key q_off + u only if bit u of the node's mask is
+          // set; nothing past L
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) {
+            const int u = j * kBN + c - kv.q_off;
+            if (u >= 0 && (u >= kv.L - kv.q_off || !((tmask >> (u & 63)) & 1ull))) s[c] = -INFINITY;
+          }
+        } else if (edge) {
           const int lim = (p.causal ? min(kv.q_off + qrow + 1, kv.L) : kv.L) - j * kBN;  // visible
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
@@ -695,7 +710,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[wg], pv_ph, abort_flag))) { ok = false; break; }
       pv_ph ^= 1;
       tc_fence_after();
-      const float inv = 1.f / lr;
+      // a row with no visible key (possible only with a tree mask) gets O = 0
+      const float inv = (kPaged && lr == 0.f) ? 0.f : 1.f / lr;
       const bool live = qrow < p.N;
       const size_t grow = static_cast<size_t>(w.bh) * p.N + qrow;
 #pragma unroll

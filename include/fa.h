@@ -180,6 +180,30 @@ fa_status fa_prefill_paged(const void *q, const void *k_pool, const void *v_pool
                            fa_stream_t stream);
 
 /*
+ * fa_tree_attention -- verification step of speculative decoding: every node of a draft-token
+ * tree is scored against the context and its own path through the tree, in one pass.
+ *
+ * The draft model proposes candidate tokens as a tree and the target model checks all of its
+ * nodes in a single forward pass with tree attention ("LLM study notes", speculative decoding).
+ * The tree's T nodes are the last T of sequence s's L = seq_lens[s] cached tokens, in topological
+ * order (their keys and values already written).  Node t sees the L - T context tokens and node u
+ * exactly when bit u of tree_mask[s * T + t] is set: its ancestors and itself for a tree, though
+ * any mask over the T nodes is accepted.  A node that sees no key at all gets O = 0 and LSE = -inf.
+ *
+ *   q            bf16 [S, H, T, d] contiguous (the nodes' queries).
+ *   k_pool, v_pool, block_table, max_blocks_per_seq, seq_lens, num_blocks, o, o_dtype, lse, d,
+ *   scale        as for fa_prefill_paged with Lq = T (each seq_lens[s] >= T).
+ *   tree_mask    uint64 [S, T], device, 8-byte aligned; must not overlap o.
+ *   T            1 .. 64.
+ * Returns FA_OK once the kernel is queued.  No workspace.
+ */
+fa_status fa_tree_attention(const void *q, const void *k_pool, const void *v_pool,
+                            const int32_t *block_table, int max_blocks_per_seq,
+                            const int32_t *seq_lens, int num_blocks, const uint64_t *tree_mask,
+                            void *o, fa_out_dtype o_dtype, float *lse, int S, int H, int T, int d,
+                            float scale, fa_stream_t stream);
+
+/*
  * fa_decode_paged_noalloc -- fa_decode_paged without a caller-supplied workspace and without any
  * allocation.  No counterpart in the paper: this is a deployment variant of the same decode step,
  * not part of the method.

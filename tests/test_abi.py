@@ -121,6 +121,17 @@ def test_bwd_workspace_and_rejections(lib):
     assert bwd(lib, ws=10 * A + 64) == 1  # workspace overlaps dV
 
 
+def test_tree_attention_rejections(lib):
+    def tree(mask=11 * A, T=8, S=2, o=7 * A, d=128):
+        return lib.fa_tree_attention(A, 2 * A, 3 * A, 5 * A, 4, 6 * A, 8, mask, o, 0, None, S, 2,
+                                     T, d, 0.0, None)
+    assert tree(mask=None) == 1
+    assert tree(T=0) == 1 and tree(T=65) == 1
+    assert tree(mask=11 * A + 4) == 3
+    assert tree(o=11 * A - 64) == 1  # output overlaps the mask
+    assert tree(d=96) == 2
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)

@@ -112,3 +112,17 @@ def test_tree_visibility_is_the_ancestor_set():
                 assert {u for u in range(40) if bits[t] >> u & 1} == anc
     with pytest.raises(ValueError):
         W.tree_visibility([0])
+
+
+def test_tree_verify_flops_counts_visible_pairs():
+    parents = [[-1, 0, 0, 1], [-1, -1, 1, 2]]
+    masks = [W.tree_visibility(p) for p in parents]
+    lens = [10, 4]
+    pairs = 0
+    for L, p in zip(lens, parents):
+        for t in range(4):
+            anc, u = 0, t
+            while u >= 0:
+                anc, u = anc + 1, p[u]
+            pairs += (L - 4) + anc
+    assert W.tree_verify_flops(lens, masks, 3, 8) == 4 * 8 * 3 * pairs

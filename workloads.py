@@ -335,6 +335,14 @@ def tree_verify_flops(lens, masks, H: int, d: int) -> int:
     return 4 * d * H * pairs
 
 
+def tree_verify_bytes(lens, H: int, d: int, T: int) -> int:
+    """Algorithmic bytes of one tree verification: K and V of every cached token (bf16), the
+    nodes' q and o (bf16), their masks (uint64), the used block-table entries and the lengths."""
+    S = len(lens)
+    pages = sum(-(-L // PAGE_SIZE) for L in lens)
+    return 2 * H * d * 2 * sum(lens) + 2 * S * H * T * d * 2 + 8 * S * T + 4 * pages + 4 * S
+
+
 def decode_bytes(lens, H: int, d: int, max_blocks: int) -> int:
     """Algorithmic bytes of one paged decode pass: K and V of every context token (bf16), q and o
     (bf16), the block-table entries actually used (int32) and the lengths (int32)."""
