@@ -41,6 +41,15 @@
  * the nodes u whose bit u is set in mask[t] (its ancestors and itself, for a tree).  A row that
  * sees no key at all has O = 0 and LSE = -inf.
  *
+ * oracle_attention_keyrange and oracle_merge_partials split one sequence's keys into ranges, as
+ * the sequence-length parallelism of "FlashAttention-2 GPU work partitioning" (section 3: a long
+ * sequence is divided among several workers) does across devices.  The partial of a key range is
+ * the plain row definition over the keys of that range the query sees (O = 0 and LSE = -inf when
+ * it sees none); partials of disjoint ranges are merged with the rescaling rule of "Flash
+ * Attention" (myungum), section 2, steps 11-12, written for log-sum-exps:
+ *     M = max_r LSE_r,  w_r = exp(LSE_r - M),  O = sum_r w_r O_r / sum_r w_r,
+ *     LSE = M + ln sum_r w_r.
+ *
  * oracle_attention_bwd is the backward pass: the gradients of the scalar sum_i dO[i] . O[i] with
  * respect to Q, K and V for a given dO.  The pages describe the backward only in prose ("Paged vs
  * Flash attention", training: gradients from the stored intermediate results, block by block;
@@ -606,5 +615,110 @@ int oracle_tree_attention(const uint16_t *q, const uint16_t *k_pool, const uint1
         pthread_join(th[t], NULL);
     free(th);
     free(jobs);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* key-range partials and their merge                                                          */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int64_t Nq, Nk, q0, k0;
+    int d, causal;
+    double scale;
+    double *o, *lse;
+    int64_t first, last; /* range of (bh, row) rows */
+} kr_job;
+
+static void *kr_worker(void *arg)
+{
+    kr_job *jb = (kr_job *)arg;
+    const int d = jb->d;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(jb->Nk > 0 ? jb->Nk : 1));
+    const uint16_t **kr = (const uint16_t **)malloc(sizeof(void *) * (size_t)(jb->Nk > 0 ? jb->Nk : 1));
+    const uint16_t **vr = (const uint16_t **)malloc(sizeof(void *) * (size_t)(jb->Nk > 0 ? jb->Nk : 1));
+    for (int64_t r = jb->first; r < jb->last; ++r) {
+        int64_t bh = r / jb->Nq, i = r % jb->Nq;
+        /* query at position q0 + i sees the range's keys at positions k0 + c <= q0 + i */
+        int64_t n_keys = jb->Nk;
+        if (jb->causal) {
+            int64_t last = jb->q0 + i - jb->k0;
+            n_keys = last < 0 ? 0 : (last + 1 < jb->Nk ? last + 1 : jb->Nk);
+        }
+        if (n_keys == 0) {
+            for (int c = 0; c < d; ++c)
+                jb->o[r * d + c] = 0.0;
+            jb->lse[r] = -INFINITY;
+            continue;
+        }
+        const uint16_t *K = jb->k + bh * jb->Nk * d, *V = jb->v + bh * jb->Nk * d;
+        for (int64_t c = 0; c < n_keys; ++c) {
+            kr[c] = K + c * d;
+            vr[c] = V + c * d;
+        }
+        const uint16_t *qi = jb->q + r * d;
+        attend_row(qi, kr, vr, n_keys, d, jb->scale, s, jb->o + r * d, jb->lse + r);
+    }
+    free(s);
+    free(kr);
+    free(vr);
+    return NULL;
+}
+
+/* q [BH, Nq, d] (positions q0 .. q0+Nq-1), k, v [BH, Nk, d] (positions k0 .. k0+Nk-1);
+ * o [BH, Nq, d], lse [BH, Nq]. */
+int oracle_attention_keyrange(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t BH,
+                              int64_t Nq, int64_t Nk, int64_t q0, int64_t k0, int d, int causal,
+                              double scale, double *o, double *lse, int nthreads)
+{
+    if (BH < 1 || Nq < 1 || Nk < 0 || d < 1 || nthreads < 1)
+        return 1;
+    int64_t rows = BH * Nq;
+    if (nthreads > rows)
+        nthreads = (int)rows;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    kr_job *jobs = (kr_job *)malloc(sizeof(kr_job) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) {
+        kr_job j = {q, k, v, Nq, Nk, q0, k0, d, causal, scale, o, lse,
+                    rows * t / nthreads, rows * (t + 1) / nthreads};
+        jobs[t] = j;
+        pthread_create(&th[t], NULL, kr_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+    free(jobs);
+    return 0;
+}
+
+/* o_parts [G, rows, d], lse_parts [G, rows] -> o [rows, d], lse [rows]. */
+int oracle_merge_partials(const double *o_parts, const double *lse_parts, int G, int64_t rows,
+                          int d, double *o, double *lse)
+{
+    if (G < 1 || rows < 0 || d < 1)
+        return 1;
+    for (int64_t r = 0; r < rows; ++r) {
+        double M = -INFINITY;
+        for (int g = 0; g < G; ++g)
+            if (lse_parts[g * rows + r] > M)
+                M = lse_parts[g * rows + r];
+        for (int c = 0; c < d; ++c)
+            o[r * d + c] = 0.0;
+        if (M == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double wsum = 0.0;
+        for (int g = 0; g < G; ++g) {
+            double w = exp(lse_parts[g * rows + r] - M);
+            wsum += w;
+            for (int c = 0; c < d; ++c)
+                o[r * d + c] += w * o_parts[(g * rows + r) * d + c];
+        }
+        for (int c = 0; c < d; ++c)
+            o[r * d + c] /= wsum;
+        lse[r] = M + log(wsum);
+    }
     return 0;
 }

@@ -59,6 +59,11 @@ class OracleLib:
                                               _int, _int, _int, _int, _int, _dbl, _f64p, _f64p,
                                               _int]
         lib.oracle_tree_attention.restype = ctypes.c_int
+        lib.oracle_attention_keyrange.argtypes = [_u16p, _u16p, _u16p, _i64, _i64, _i64, _i64,
+                                                  _i64, _int, _int, _dbl, _f64p, _f64p, _int]
+        lib.oracle_attention_keyrange.restype = ctypes.c_int
+        lib.oracle_merge_partials.argtypes = [_f64p, _f64p, _int, _i64, _int, _f64p, _f64p]
+        lib.oracle_merge_partials.restype = ctypes.c_int
         lib.oracle_attention_bwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _i64, _int, _int, _dbl,
                                              _i64p, _i64, _f64p, _f64p, _f64p, _int]
         for f in (lib.oracle_attention, lib.oracle_attention_rows, lib.oracle_attention_probs,
@@ -115,6 +120,36 @@ class OracleLib:
         if rc:
             raise ValueError("oracle_flash_alg1: bad arguments")
         return O, l, m
+
+    def attention_keyrange(self, q, k, v, q0: int, k0: int, causal: bool, scale: float,
+                           nthreads: int | None = None):
+        """Partial attention of queries at positions q0.. over keys at positions k0.. of the same
+        sequences.  q [..., Nq, d], k, v [..., Nk, d] (uint16 bf16 bits).  Rows that see no key
+        get O = 0, LSE = -inf.  Returns (o [..., Nq, d], lse [..., Nq])."""
+        q, k, v = _bits(q), _bits(k), _bits(v)
+        *lead, Nq, d = q.shape
+        Nk = k.shape[-2]
+        BH = int(np.prod(lead)) if lead else 1
+        o = np.empty((BH, Nq, d), np.float64)
+        lse = np.empty((BH, Nq), np.float64)
+        rc = self.lib.oracle_attention_keyrange(q, k, v, BH, Nq, Nk, q0, k0, d, int(causal), scale,
+                                                o, lse, nthreads or default_threads())
+        if rc:
+            raise ValueError("oracle_attention_keyrange: bad arguments")
+        return o.reshape(*lead, Nq, d), lse.reshape(*lead, Nq)
+
+    def merge_partials(self, o_parts, lse_parts):
+        """o_parts [G, ..., d], lse_parts [G, ...] (float64).  Returns the merged (o, lse)."""
+        o_parts = np.ascontiguousarray(o_parts, dtype=np.float64)
+        lse_parts = np.ascontiguousarray(lse_parts, dtype=np.float64)
+        G, d = o_parts.shape[0], o_parts.shape[-1]
+        rows = int(np.prod(o_parts.shape[1:-1]))
+        o = np.empty(o_parts.shape[1:], np.float64)
+        lse = np.empty(lse_parts.shape[1:], np.float64)
+        rc = self.lib.oracle_merge_partials(o_parts, lse_parts, G, rows, d, o, lse)
+        if rc:
+            raise ValueError("oracle_merge_partials: bad arguments")
+        return o, lse
 
     def tree_attention(self, q, k_pool, v_pool, block_table, seq_lens, tree_mask, scale: float,
                        page: int = 16, nthreads: int | None = None):
@@ -242,3 +277,11 @@ def attention_bwd(*a, **kw):
 
 def tree_attention(*a, **kw):
     return default().tree_attention(*a, **kw)
+
+
+def attention_keyrange(*a, **kw):
+    return default().attention_keyrange(*a, **kw)
+
+
+def merge_partials(*a, **kw):
+    return default().merge_partials(*a, **kw)

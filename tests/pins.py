@@ -15,6 +15,9 @@ The facts used:
   block sizes give the plain result;
 * a paged KV cache is only a relocation of logically contiguous rows ("LLM study notes", paged
   attention);
+* a sequence's keys can be split into ranges whose partial results merge with the tiled
+  algorithm's rescaling rule ("FlashAttention-2 GPU work partitioning", section 3; "Flash
+  Attention" (myungum), section 2);
 * a draft-token tree is verified in one pass, each node continuing the context along its path
   ("LLM study notes", speculative decoding), so a node sees its ancestors and itself;
 * the backward pass returns the gradients of sum(dO * O) with respect to Q, K and V (the pages
@@ -452,8 +455,59 @@ def pin_tree_attention(orc):
     assert np.all(np.isneginf(lse[0, :, 4])), "empty row: LSE = -inf"
 
 
+def pin_key_ranges_merge(orc):
+    """Splitting the keys into ranges and merging the range partials gives plain attention, for
+    any split (sequence-length parallelism; the merge is the rescaling rule of the tiled
+    algorithm); a range partial is scipy's softmax over that range's visible keys; an empty
+    partial (O = 0, LSE = -inf) changes nothing; the merge of log-sum-exps near 1000 stays finite
+    and equals scipy's logsumexp."""
+    BH, N, d, scale = 2, 70, 16, 0.3
+    q, k, v = (rnd((BH, N, d), 120 + t) for t in range(3))
+    for causal in (False, True):
+        full_o, full_l = orc.attention(q, k, v, causal, scale)
+        for cuts in ([35], [1, 69], [10, 30, 31, 60], [70]):
+            bounds = [0] + cuts + ([N] if cuts[-1] != N else [])
+            parts_o, parts_l = [], []
+            for a, b in zip(bounds[:-1], bounds[1:]):
+                po, pl = orc.attention_keyrange(q, k[:, a:b].copy(), v[:, a:b].copy(), 0, a, causal,
+                                                scale)
+                parts_o.append(po)
+                parts_l.append(pl)
+            mo, ml = orc.merge_partials(np.stack(parts_o), np.stack(parts_l))
+            close(mo, full_o, 1e-13, f"merged key ranges {cuts} causal={causal}")
+            close(ml, full_l, 1e-13, f"merged key ranges LSE {cuts} causal={causal}")
+        # one middle range against scipy, queries at positions 40.. over keys at 20..50
+        po, pl = orc.attention_keyrange(q[:, 40:].copy(), k[:, 20:50].copy(), v[:, 20:50].copy(), 40,
+                                        20, causal, scale)
+        for h in range(BH):
+            S_ = scale * widen(q[h, 40:]) @ widen(k[h, 20:50]).T
+            if causal:
+                for i in range(N - 40):
+                    S_[i, (40 + i) - 20 + 1:] = -np.inf
+            close(po[h], sps.softmax(S_, axis=1) @ widen(v[h, 20:50]), 1e-13, "range partial O")
+            close(pl[h], sps.logsumexp(S_, axis=1), 1e-13, "range partial LSE")
+    # causal: queries before the range see nothing
+    po, pl = orc.attention_keyrange(q, k[:, 50:].copy(), v[:, 50:].copy(), 0, 50, True, scale)
+    close(po[:, :50], np.zeros((BH, 50, d)), 0.0, "no visible key: O = 0")
+    assert np.all(np.isneginf(pl[:, :50])), "no visible key: LSE = -inf"
+    # neutrality of an empty partial
+    o1, l1 = orc.attention(q, k, v, False, scale)
+    mo, ml = orc.merge_partials(np.stack([o1, np.zeros_like(o1)]),
+                                np.stack([l1, np.full_like(l1, -np.inf)]))
+    close(mo, o1, 0.0, "empty partial is neutral")
+    close(ml, l1, 0.0, "empty partial is neutral LSE")
+    # large log-sum-exps: exact reference from scipy's logsumexp on the weights
+    rng = np.random.default_rng(7)
+    lp = 1000.0 + rng.normal(size=(3, 5))
+    op = rng.normal(size=(3, 5, 4))
+    mo, ml = orc.merge_partials(op, lp)
+    w = np.exp(lp - sps.logsumexp(lp, axis=0))
+    close(mo, np.einsum("gr,grc->rc", w, op), 1e-12, "merge weights at LSE ~ 1000")
+    close(ml, sps.logsumexp(lp, axis=0), 1e-12, "merged LSE at ~ 1000")
+
+
 ALL_PINS = [pin_uniform_scores, pin_single_key, pin_dominant_score, pin_two_keys_logistic,
             pin_shift_invariance, pin_rows_sum_to_one, pin_library_softmax, pin_permutation,
             pin_linear_in_v, pin_tiled_algorithm, pin_paged_decode, pin_paged_prefill,
             pin_bwd_finite_differences, pin_bwd_autograd, pin_bwd_closed_forms,
-            pin_tree_attention]
+            pin_tree_attention, pin_key_ranges_merge]

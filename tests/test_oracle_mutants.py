@@ -54,6 +54,10 @@ MUTANTS = {
     "tree_offset": ("int64_t L = jb->lens[sq], ctx = L - T;", "int64_t L = jb->lens[sq], ctx = L - T + 1;"),
     "tree_bit_order": ("if (key >= ctx && !((m >> (key - ctx)) & 1u))",
                        "if (key >= ctx && !((m >> (T - 1 - (key - ctx))) & 1u))"),
+    "range_causal_offset": ("int64_t last = jb->q0 + i - jb->k0;", "int64_t last = jb->q0 + i - jb->k0 - 1;"),
+    "merge_weight_sign": ("double w = exp(lse_parts[g * rows + r] - M);", "double w = exp(M - lse_parts[g * rows + r]);"),
+    "merge_no_shift": ("double w = exp(lse_parts[g * rows + r] - M);", "double w = exp(lse_parts[g * rows + r]);"),
+    "merge_lse_no_log": ("lse[r] = M + log(wsum);", "lse[r] = M + wsum;"),
 }
 
 
