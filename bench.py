@@ -16,7 +16,8 @@ oracle on this host's cores, a bounded row sample), `e2e` (the same metric throu
 with Q/K/V copied from pinned host memory and O/LSE copied back inside the timed region), `sweep`
 (the sequence-length grid, d = 128 and d = 64), `decode` (paged decode GB/s vs HBM),
 `paged_prefill` (chunked prefill through the block table, TFLOP/s), `backward` (fa_bwd TFLOP/s),
-`tree` (draft-tree verification TFLOP/s) and `clocks`.
+`tree` (draft-tree verification TFLOP/s), `sequence_parallel` (one long sequence with its keys
+split over ranks: partials, all-gather, merge) and `clocks`.
 """
 from __future__ import annotations
 
@@ -320,6 +321,69 @@ def bench_tree(fa, args, dev, flush, stream, pk):
             "launches_per_step": 1}
 
 
+def bench_sequence_parallel(fa, args, dev, flush, stream, pk, rank, world):
+    """One long causal sequence, B1 H16 N32768 d128, with its keys split into contiguous ranges.
+    With N GPUs each rank holds one range: partial of every query over it (fa_fwd_keyrange), an
+    NCCL all-gather of the partials, and the merge (fa_merge_partials) on every rank.  On one GPU
+    the four ranges of a 4-way split run one after another before the same merge."""
+    from exact_attention_158_b200 import sequence_parallel as sp
+    case = W.PrefillCase("seqpar", 1, 16, 32768, 128, True)
+    q, k, v = W.make_prefill(case, device=dev)
+    G = world if world > 1 else 4
+    ranges = sp.key_ranges(case.N, G)
+    mine = [ranges[rank]] if world > 1 else ranges
+    shards = [(a, k[:, :, a:b].contiguous(), v[:, :, a:b].contiguous()) for a, b in mine]
+    del k, v
+    o_all = torch.empty((G, *q.shape), dtype=torch.float32, device=dev)
+    l_all = torch.empty((G, *q.shape[:3]), dtype=torch.float32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    lib = fa.load_library()
+    st = stream.cuda_stream
+
+    def merge():
+        rc = lib.fa_merge_partials(o_all.data_ptr(), l_all.data_ptr(), G, lse.numel(), case.d,
+                                   o.data_ptr(), 0, lse.data_ptr(), st)
+        if rc != 0:
+            raise RuntimeError(f"fa_merge_partials: {rc}")
+
+    def step():
+        if world > 1:
+            a, ks, vs = shards[0]
+            fa.fa_fwd_keyrange(q, ks, vs, k_pos0=a, causal=True, out=o_all[rank], lse=l_all[rank])
+            # in place: this rank's slice of the gathered buffer is its input
+            torch.distributed.all_gather_into_tensor(o_all, o_all[rank])
+            torch.distributed.all_gather_into_tensor(l_all, l_all[rank])
+        else:
+            for r, (a, ks, vs) in enumerate(shards):
+                fa.fa_fwd_keyrange(q, ks, vs, k_pos0=a, causal=True, out=o_all[r], lse=l_all[r])
+        merge()
+
+    torch.cuda.nvtx.range_push("bench_sequence_parallel_timed")
+    ts = time_launches(step, args.sweep_steps, 3, flush, stream)
+    merge_ts = time_launches(merge, args.sweep_steps, 3, flush, stream)
+    torch.cuda.nvtx.range_pop()
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during the sequence-parallel bench")
+    ms = dist_max(statistics.median(ts))
+    mms = dist_max(statistics.median(merge_ts))
+    tf = case.flops / (ms * 1e-3) / 1e12
+    rows = lse.numel()
+    merge_bytes = G * rows * (case.d + 1) * 4 + rows * case.d * 2 + rows * 4
+    mgbs = merge_bytes / (mms * 1e-3) / 1e9
+    return {"metric": "sequence-sharded causal forward TFLOP/s (whole sequence, all ranks)",
+            "workload": "B1 H16 N32768 d128 causal, keys and values split into contiguous ranges",
+            "ranges": G, "emulated_on_one_gpu": world == 1,
+            "ms": round(ms, 4), "value": round(tf, 1), "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                         "peak": pk["bf16_tflops"] * (world if world > 1 else 1), "unit": "TFLOP/s",
+                         "frac": round(tf / (pk["bf16_tflops"] * (world if world > 1 else 1)), 4)},
+            "merge": {"ms": round(mms, 4), "algorithmic_bytes": merge_bytes,
+                      "roofline": {"bound": "hbm", "achieved": round(mgbs, 1), "peak": pk["hbm_gbs"],
+                                   "unit": "GB/s", "frac": round(mgbs / pk["hbm_gbs"], 4)}},
+            "launches_per_step": (1 if world > 1 else G) + 1}
+
+
 def bench_backward(fa, args, dev, flush, stream, pk):
     """fa_bwd on the headline shape (B8 H16 N2048 d128), non-causal and causal.  FLOPs are the five
     matmuls per (query, key) pair: 2.5x the forward's 4 B H N^2 d (halved causal)."""
@@ -362,6 +426,10 @@ def bench_ours(args, rank, world):
         return {"metric": METRIC, "decode": bench_decode(fa, args, dev, flush, stream, pk)}
     if args.only == "tree":
         return {"metric": METRIC, "tree": bench_tree(fa, args, dev, flush, stream, pk)}
+    if args.only == "seqpar":
+        return {"metric": METRIC,
+                "sequence_parallel": bench_sequence_parallel(fa, args, dev, flush, stream, pk,
+                                                             rank, world)}
     if args.only == "backward":
         return {"metric": METRIC, "backward": bench_backward(fa, args, dev, flush, stream, pk)}
     if args.only == "paged":
@@ -491,8 +559,12 @@ def bench_ours(args, rank, world):
     # ---- draft-tree verification (tensor bound, short query tiles)
     tree = None if args.no_tree else bench_tree(fa, args, dev, flush, stream, pk)
 
+    # ---- sequence-sharded forward (partials + merge; ranks emulated on one GPU)
+    seqpar = (None if args.no_seqpar else
+              bench_sequence_parallel(fa, args, dev, flush, stream, pk, rank, world))
+
     result.update({"e2e": e2e, "sweep": sweep, "decode": dec, "paged_prefill": paged,
-                   "backward": bwd, "tree": tree})
+                   "backward": bwd, "tree": tree, "sequence_parallel": seqpar})
     return result
 
 
@@ -528,10 +600,12 @@ def main():
     ap.add_argument("--no-paged", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-tree", action="store_true")
+    ap.add_argument("--no-seqpar", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="sequences in the decode workload (64 is the benchmark; fewer for profiling)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "paged", "backward", "tree"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "paged", "backward", "tree",
+                                       "seqpar"],
                     default="all",
                     help="prefill: the headline loop alone; decode / paged: the paged decode or "
                     "chunked prefill loop alone")

@@ -18,7 +18,7 @@ import torch
 from . import build as _build
 
 __all__ = ["fa_fwd", "fa_bwd", "fa_decode_paged", "fa_decode_paged_noalloc", "fa_prefill_paged",
-           "fa_tree_attention",
+           "fa_tree_attention", "fa_fwd_keyrange", "fa_merge_partials",
            "fa_decode_workspace_size",
            "NOALLOC_SCRATCH_BYTES", "device_status",
            "FaError", "library_path", "load_library", "EXPORTED_SYMBOLS", "STATUS"]
@@ -29,6 +29,7 @@ FA_OUT_BF16, FA_OUT_F32 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
                     "fa_decode_paged_noalloc", "fa_prefill_paged", "fa_tree_attention",
+                    "fa_fwd_keyrange", "fa_merge_partials",
                     "fa_bwd_workspace_size",
                     "fa_bwd", "fa_get_device_status",
                     "fa_status_string",
@@ -73,6 +74,11 @@ def load_library():
     lib.fa_prefill_paged.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, i32, vp, i32, i32, i32, i32,
                                      i32, f32, vp]
     lib.fa_prefill_paged.restype = i32
+    lib.fa_fwd_keyrange.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32,
+                                    i32, f32, vp]
+    lib.fa_fwd_keyrange.restype = i32
+    lib.fa_merge_partials.argtypes = [vp, vp, i32, ctypes.c_longlong, i32, vp, i32, vp, vp]
+    lib.fa_merge_partials.restype = i32
     lib.fa_tree_attention.argtypes = [vp, vp, vp, vp, i32, vp, i32, vp, vp, i32, vp, i32, i32, i32,
                                       i32, f32, vp]
     lib.fa_tree_attention.restype = i32
@@ -226,6 +232,52 @@ def fa_bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = No
                         _stream_handle(stream))
     _check(st, "fa_bwd")
     return dq, dk, dv
+
+
+def fa_fwd_keyrange(q, k, v, q_row0: int = 0, k_pos0: int = 0, causal: bool = False,
+                    scale: float | None = None, out_dtype=torch.float32, out=None, lse=None,
+                    stream=None):
+    """Partial attention of the query rows q_row0.. of q [B, H, Nq, d] (row i at position i) over
+    the keys k, v [B, H, Nk, d] at positions k_pos0...  Rows that see no key get O = 0,
+    LSE = -inf; rows before q_row0 of out / lse are left as they are.  Returns (o, lse)."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if k.shape != (B, H, Nk, d) or v.shape != k.shape:
+        raise ValueError("k, v must be [B, H, Nk, d] with q's B, H, d")
+    code = _out_code(out_dtype)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib.fa_fwd_keyrange(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), code,
+                                 lse.data_ptr(), B, H, Nq, q_row0, Nk, k_pos0, d, int(causal),
+                                 float(scale) if scale is not None else 0.0, _stream_handle(stream))
+    _check(st, "fa_fwd_keyrange")
+    return out, lse
+
+
+def fa_merge_partials(o_parts, lse_parts, out_dtype=torch.bfloat16, stream=None):
+    """o_parts fp32 [G, ..., d], lse_parts fp32 [G, ...]: partials of the same rows over disjoint
+    key ranges.  Returns the merged (o [..., d], lse [...])."""
+    lib = load_library()
+    _require(o_parts, "o_parts", torch.float32)
+    _require(lse_parts, "lse_parts", torch.float32)
+    G, d = o_parts.shape[0], o_parts.shape[-1]
+    if lse_parts.shape != o_parts.shape[:-1]:
+        raise ValueError("lse_parts must be o_parts' shape without the last dimension")
+    rows = lse_parts[0].numel()
+    code = _out_code(out_dtype)
+    o = torch.empty(o_parts.shape[1:], dtype=out_dtype, device=o_parts.device)
+    lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    with torch.cuda.device(o_parts.device):
+        st = lib.fa_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), G, rows, d,
+                                   o.data_ptr(), code, lse.data_ptr(), _stream_handle(stream))
+    _check(st, "fa_merge_partials")
+    return o, lse
 
 
 def fa_tree_attention(q, k_pool, v_pool, block_table, seq_lens, tree_mask,

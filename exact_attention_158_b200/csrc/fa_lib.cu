@@ -1,10 +1,11 @@
 // fa_lib.cu -- the C ABI declared in include/fa.h: argument checks, TMA descriptors, launches.
 // Host code only decides shapes and launches; every step of the attention itself runs in the
-// kernels of fa_prefill.cuh, fa_backward.cuh and fa_decode.cuh.
+// kernels of fa_prefill.cuh, fa_backward.cuh, fa_decode.cuh and fa_merge.cuh.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -15,6 +16,7 @@
 #include "fa.h"
 #include "fa_backward.cuh"
 #include "fa_decode.cuh"
+#include "fa_merge.cuh"
 #include "fa_prefill.cuh"
 
 namespace fa {
@@ -46,7 +48,7 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int num_sms = 0;
-  bool prefill_attr[4] = {false, false, false, false};  // (d = 64, 128) x (contiguous, paged)
+  bool prefill_attr[6] = {};  // (d = 64, 128) x (square, paged, key range)
   bool bwd_attr[2] = {false, false};                    // d = 64, 128
 };
 
@@ -152,17 +154,17 @@ bool encode_pool(CUtensorMap *map, const void *base, int d, int H, int num_block
   return r == CUDA_SUCCESS;
 }
 
-template <int HD, bool kPaged>
+template <int HD, int kMode>
 fa_status launch_prefill(DeviceInfo &dev, const CUtensorMap &tq, const CUtensorMap &tk,
                          const CUtensorMap &tv, fa::PrefillParams p, cudaStream_t stream) {
   using C = fa::PrefillCfg<HD>;
   p.num_pairs = (p.N + 2 * fa::kBM - 1) / (2 * fa::kBM);
   p.num_units = p.BH * p.num_pairs;
-  const int slot = (HD == 128 ? 1 : 0) + (kPaged ? 2 : 0);
+  const int slot = (HD == 128 ? 1 : 0) + 2 * kMode;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!dev.prefill_attr[slot]) {
-      cudaError_t e = cudaFuncSetAttribute(fa::fa_prefill_kernel<HD, kPaged>,
+      cudaError_t e = cudaFuncSetAttribute(fa::fa_prefill_kernel<HD, kMode>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(C::kSmemBytes));
       if (e != cudaSuccess) return launch_failed(e);
@@ -170,7 +172,7 @@ fa_status launch_prefill(DeviceInfo &dev, const CUtensorMap &tq, const CUtensorM
     }
   }
   const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
-  fa::fa_prefill_kernel<HD, kPaged><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk,
+  fa::fa_prefill_kernel<HD, kMode><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk,
                                                                                          tv, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : launch_failed(e);
@@ -194,7 +196,9 @@ fa_status launch_prefill_dense(DeviceInfo &dev, const void *q, const void *k, co
   p.N = N;
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
-  return launch_prefill<HD, false>(dev, tq, tk, tv, p, stream);
+  p.q_rows = N;
+  p.Nk = N;
+  return launch_prefill<HD, fa::kModeSquare>(dev, tq, tk, tv, p, stream);
 }
 
 // Backward workspace: dQ accumulator fp32 [BH, Np, d], then LSE2 and D fp32 [BH, Np] each, with
@@ -584,8 +588,9 @@ static fa_status prefill_paged_impl(const void *q, const void *k_pool, const voi
   p.H = H;
   p.tree_mask = tree_mask;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 128) return launch_prefill<128, true>(*dev, tq, tk, tv, p, s);
-  return launch_prefill<64, true>(*dev, tq, tk, tv, p, s);
+  p.q_rows = Lq;
+  if (d == 128) return launch_prefill<128, fa::kModePaged>(*dev, tq, tk, tv, p, s);
+  return launch_prefill<64, fa::kModePaged>(*dev, tq, tk, tv, p, s);
 }
 
 fa_status fa_prefill_paged(const void *q, const void *k_pool, const void *v_pool,
@@ -613,6 +618,102 @@ fa_status fa_tree_attention(const void *q, const void *k_pool, const void *v_poo
   }
   return prefill_paged_impl(q, k_pool, v_pool, block_table, max_blocks_per_seq, seq_lens,
                             num_blocks, tree_mask, o, o_dtype, lse, S, H, T, d, 0, scale, stream);
+}
+
+fa_status fa_fwd_keyrange(const void *q, const void *k, const void *v, void *o, fa_out_dtype o_dtype,
+                          float *lse, int B, int H, int Nq, int q_row0, int Nk, int k_pos0, int d,
+                          int causal, float scale, fa_stream_t stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || q_row0 < 0 || q_row0 >= Nq || k_pos0 < 0)
+    return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  float sc;
+  if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  const int BH = B * H;
+  const size_t qrows = static_cast<size_t>(BH) * Nq, krows = static_cast<size_t>(BH) * Nk;
+  const size_t o_bytes = qrows * d * (o_dtype == FA_OUT_F32 ? 4 : 2);
+  if (overlaps(o, o_bytes, q, qrows * d * 2) || overlaps(o, o_bytes, k, krows * d * 2) ||
+      overlaps(o, o_bytes, v, krows * d * 2))
+    return FA_ERR_INVALID_ARG;
+  if (lse && (overlaps(lse, qrows * 4, o, o_bytes) || overlaps(lse, qrows * 4, q, qrows * d * 2)))
+    return FA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int o_f32 = o_dtype == FA_OUT_F32;
+  // causal: rows before the range's first key see none of it
+  const int q_start = causal ? std::max(q_row0, std::min(k_pos0, Nq)) : q_row0;
+  if (q_start > q_row0) {
+    const long long threads = static_cast<long long>(BH) * (q_start - q_row0) * (d / 4);
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    if (d == 128)
+      fa::fa_empty_rows_kernel<128><<<blocks, 256, 0, s>>>(o, o_f32, lse, BH, Nq, q_row0, q_start);
+    else
+      fa::fa_empty_rows_kernel<64><<<blocks, 256, 0, s>>>(o, o_f32, lse, BH, Nq, q_row0, q_start);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return launch_failed(e);
+  }
+  if (q_start >= Nq) return FA_OK;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bhnd(&tq, q, d, Nq, BH) || !encode_bhnd(&tk, k, d, Nk, BH) ||
+      !encode_bhnd(&tv, v, d, Nk, BH)) {
+    t_last_error = "cuTensorMapEncodeTiled failed";
+    return FA_ERR_LAUNCH;
+  }
+  fa::PrefillParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.o_f32 = o_f32;
+  p.BH = BH;
+  p.N = Nq - q_start;
+  p.causal = causal;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.q_row0 = q_start;
+  p.q_rows = Nq;
+  p.Nk = Nk;
+  p.q_off = causal ? q_start - k_pos0 : 0;
+  if (d == 128) return launch_prefill<128, fa::kModeRange>(*dev, tq, tk, tv, p, s);
+  return launch_prefill<64, fa::kModeRange>(*dev, tq, tk, tv, p, s);
+}
+
+fa_status fa_merge_partials(const float *o_parts, const float *lse_parts, int G, long long rows,
+                            int d, void *o, fa_out_dtype o_dtype, float *lse, fa_stream_t stream) {
+  if (!o_parts || !lse_parts || !o) return FA_ERR_INVALID_ARG;
+  if (G < 1 || rows < 1) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (rows > (1ll << 40) / d) return FA_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  const size_t o_bytes = static_cast<size_t>(rows) * d * (o_dtype == FA_OUT_F32 ? 4 : 2);
+  const size_t parts_bytes = static_cast<size_t>(G) * rows * d * 4;
+  if (overlaps(o, o_bytes, o_parts, parts_bytes) ||
+      overlaps(o, o_bytes, lse_parts, static_cast<size_t>(G) * rows * 4))
+    return FA_ERR_INVALID_ARG;
+  if (lse && (overlaps(lse, rows * 4, o_parts, parts_bytes) || overlaps(lse, rows * 4, o, o_bytes)))
+    return FA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long threads = rows * (d / 4);
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  const int o_f32 = o_dtype == FA_OUT_F32;
+  if (d == 128)
+    fa::fa_merge_kernel<128><<<blocks, 256, 0, s>>>(o_parts, lse_parts, G, rows, o, o_f32, lse);
+  else
+    fa::fa_merge_kernel<64><<<blocks, 256, 0, s>>>(o_parts, lse_parts, G, rows, o, o_f32, lse);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : launch_failed(e);
 }
 
 fa_status fa_get_device_status(fa_stream_t stream) {

@@ -71,7 +71,7 @@ struct PrefillParams {
   void *o;
   float *lse;
   int o_f32;
-  int BH, N, causal;  // N: query rows per (b, h); also the key count unless paged
+  int BH, N, causal;  // N: query rows per (b, h) processed; also the key count in the square mode
   float scale_log2;   // scale * log2(e)
   int num_pairs;      // ceil(N / 256)
   int num_units;      // BH * num_pairs query-tile pairs, scheduled over the persistent CTAs
@@ -84,7 +84,16 @@ struct PrefillParams {
   // the last N cached tokens in topological order; bit u of tree_mask[s * N + t] set when node t
   // sees node u (N <= 64).  Null otherwise.
   const uint64_t *tree_mask;
+  // key-range mode: the processed queries are rows q_row0 .. q_row0 + N - 1 of Q / O / LSE tensors
+  // with q_rows rows per (b, h); the keys are the Nk rows of K / V; query row r sits at key
+  // position q_off + r (>= 0).  The other modes use q_row0 = 0 and q_rows = N.
+  int q_row0, q_rows, Nk, q_off;
 };
+
+// Kernel modes: square prefill (keys = queries), paged cache (keys gathered through the block
+// table, queries the last N of each sequence), key range (contiguous keys of one range of the
+// sequence, queries a suffix of the query rows).
+constexpr int kModeSquare = 0, kModePaged = 1, kModeRange = 2;
 
 // Key count of unit (b, h) and the position of its first query among the keys.
 struct KvSpan {
@@ -92,9 +101,11 @@ struct KvSpan {
   int q_off;  // query row r sits at key position q_off + r
 };
 
-template <bool kPaged>
+template <int kMode>
 __device__ __forceinline__ KvSpan kv_span(const PrefillParams &p, int bh) {
-  if constexpr (kPaged) {
+  if constexpr (kMode == kModeRange) {
+    return {p.Nk, p.q_off};
+  } else if constexpr (kMode == kModePaged) {
     int L = p.seq_lens[bh / p.H];
     const int hi = p.max_blocks * 16;
     L = L < p.N ? p.N : (L > hi ? hi : L);  // out-of-contract lengths are clamped, not trusted
@@ -117,8 +128,8 @@ struct WorkUnit {
 };
 
 // The unit CTA blockIdx.x processes in its round r, or -1 once it has none left.
-// (Paged units are numbered head-major like non-causal ones: their costs depend on the device-side
-// sequence lengths, which the host does not see.)
+// (Paged and key-range units are numbered head-major like non-causal ones: their costs depend on
+// per-unit spans that the longest-first order does not model.)
 template <bool kPaged = false>
 __device__ __forceinline__ int unit_for_round(const PrefillParams &p, int r) {
   const int G = gridDim.x, c = blockIdx.x;
@@ -145,7 +156,8 @@ __device__ __forceinline__ int tile_blocks(const PrefillParams &p, const KvSpan 
   const int q0 = pr * 2 * kBM + i * kBM;
   if (q0 >= p.N) return 0;
   if (!p.causal) return (kv.L + kBN - 1) / kBN;
-  const int last_key = kv.q_off + min(q0 + kBM, p.N) - 1;
+  // (the key-range mode may have more queries than keys: clamp to the last key)
+  const int last_key = min(kv.q_off + min(q0 + kBM, p.N) - 1, kv.L - 1);
   return last_key / kBN + 1;
 }
 
@@ -260,14 +272,16 @@ __device__ __forceinline__ void store_p_row(uint8_t *p_tile, int row, const uint
   }
 }
 
-// kPaged: keys and values come from a paged cache (tm_k / tm_v are 4-D maps over the pools
-// [num_blocks, H, 16, d]; a 128-key tile is gathered as eight 16-row pages through the block table).
-template <int HD, bool kPaged>
+// kMode: kModeSquare, kModePaged (tm_k / tm_v are 4-D maps over the pools [num_blocks, H, 16, d];
+// a 128-key tile is gathered as eight 16-row pages through the block table) or kModeRange.
+template <int HD, int kMode>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
   using C = PrefillCfg<HD>;
+  constexpr bool kPaged = kMode == kModePaged;
+  constexpr bool kGeneral = kMode != kModeSquare;  // key count and query offset per unit
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -370,11 +384,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         return true;
       };
       for (int r = 0; ok; ++r) {
-        const int u = unit_for_round<kPaged>(p, r);
+        const int u = unit_for_round<kGeneral>(p, r);
         if (u < 0) break;
-        const WorkUnit w = decode_unit<kPaged>(p, u);
+        const WorkUnit w = decode_unit<kGeneral>(p, u);
         const int pr = w.pair;
-        const KvSpan kv = kv_span<kPaged>(p, w.bh);
+        const KvSpan kv = kv_span<kMode>(p, w.bh);
         kv_len = kv.L;
         if (kPaged && p.seq_lens[w.bh / p.H] != kv.L)
           atomicExch(&g_device_status, 1 /* FA_ERR_INVALID_ARG: length outside [Lq, 16*max_blocks] */);
@@ -388,7 +402,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if ((i == 0 ? n0 : n1) == 0) continue;
           for (int ch = 0; ch < C::kChunks; ++ch)
             tma_load_3d(sQ + i * C::kTileBytes + ch * C::kChunkBytes, &tm_q, q_full, ch * 64,
-                        pr * 2 * kBM + i * kBM, w.bh);
+                        (kGeneral ? p.q_row0 : 0) + pr * 2 * kBM + i * kBM, w.bh);
         }
         if (!load_kv(&tm_k, 0, w.bh)) { ok = false; break; }
         for (int j = 0; ok && j < nmax; ++j) {
@@ -423,11 +437,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
         bool ok = true;
         for (int r = 0; ok; ++r) {
-          const int u = unit_for_round<kPaged>(p, r);
+          const int u = unit_for_round<kGeneral>(p, r);
           if (u < 0) break;
-          const WorkUnit w = decode_unit<kPaged>(p, u);
+          const WorkUnit w = decode_unit<kGeneral>(p, u);
           const int pr = w.pair;
-          const KvSpan kv = kv_span<kPaged>(p, w.bh);
+          const KvSpan kv = kv_span<kMode>(p, w.bh);
           const int n[2] = {tile_blocks(p, kv, pr, 0), tile_blocks(p, kv, pr, 1)};
           const int nmax = n[0] > n[1] ? n[0] : n[1];
           if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
@@ -521,11 +535,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           return true;
         };
         for (int r = 0; ok; ++r) {
-          const int u = unit_for_round<kPaged>(p, r);
+          const int u = unit_for_round<kGeneral>(p, r);
           if (u < 0) break;
-          const WorkUnit w = decode_unit<kPaged>(p, u);
+          const WorkUnit w = decode_unit<kGeneral>(p, u);
           const int pr = w.pair;
-          const KvSpan kv = kv_span<kPaged>(p, w.bh);
+          const KvSpan kv = kv_span<kMode>(p, w.bh);
           const int n[2] = {tile_blocks(p, kv, pr, 0), tile_blocks(p, kv, pr, 1)};
           const int nmax = n[0] > n[1] ? n[0] : n[1];
           if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
@@ -589,11 +603,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t s_ph = 0, pv_ph = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-      const int u = unit_for_round<kPaged>(p, r);
+      const int u = unit_for_round<kGeneral>(p, r);
       if (u < 0) break;
-      const WorkUnit w = decode_unit<kPaged>(p, u);
+      const WorkUnit w = decode_unit<kGeneral>(p, u);
       const int pr = w.pair;
-      const KvSpan kv = kv_span<kPaged>(p, w.bh);
+      const KvSpan kv = kv_span<kMode>(p, w.bh);
       const int n = tile_blocks(p, kv, pr, wg);
       if (n == 0) continue;
       const int qrow = pr * 2 * kBM + wg * kBM + row;
@@ -619,7 +633,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // masking only where a block reaches past this tile's first row's last visible key or
         // past the last key
         bool edge;
-        if constexpr (kPaged)
+        if constexpr (kGeneral)
           edge = (p.causal && (j + 1) * kBN - 1 > kv.q_off + pr * 2 * kBM + wg * kBM) ||
                  ((j + 1) * kBN > kv.L) || (tree && (j + 1) * kBN > kv.q_off);
         else  // q_off = 0, L = N: only a causal tile's diagonal block and a ragged last block
@@ -713,7 +727,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // a row with no visible key (possible only with a tree mask) gets O = 0
       const float inv = (kPaged && lr == 0.f) ? 0.f : 1.f / lr;
       const bool live = qrow < p.N;
-      const size_t grow = static_cast<size_t>(w.bh) * p.N + qrow;
+      const size_t grow = kGeneral ? static_cast<size_t>(w.bh) * p.q_rows + p.q_row0 + qrow
+                                   : static_cast<size_t>(w.bh) * p.N + qrow;
 #pragma unroll
       for (int cc = 0; cc < HD; cc += 32) {
         uint32_t o[32];

@@ -75,6 +75,43 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, fa_out_dt
                  fa_stream_t stream);
 
 /*
+ * fa_fwd_keyrange -- attention of queries over one contiguous range of the same sequence's keys:
+ * the partial that one device computes when a long sequence's keys and values are split across
+ * devices (sequence-length parallelism, "FlashAttention-2 GPU work partitioning", section 3).
+ *
+ * Query row i of q (i in [q_row0, Nq)) sits at position i; key row c of k, v sits at position
+ * k_pos0 + c.  causal = 1: a query sees the keys at positions <= its own; otherwise all Nk keys.
+ * O and LSE are those of the plain row definition over the keys each query sees (normalised
+ * within the range); a row that sees none of them gets O = 0 and LSE = -inf.  Rows < q_row0 of o
+ * and lse are not touched.  Partials of disjoint ranges combine with fa_merge_partials.
+ *
+ *   q            bf16 [B, H, Nq, d];  k, v: bf16 [B, H, Nk, d];  16-byte aligned.
+ *   o            [B, H, Nq, d], bf16 or fp32 per o_dtype (fp32 for partials to be merged);
+ *                lse: fp32 [B, H, Nq] or NULL (needed for merging).  Must not overlap the inputs.
+ *   B, H, Nq, Nk >= 1;  0 <= q_row0 < Nq;  k_pos0 >= 0;  d: 64 or 128;  causal 0/1;  scale as for
+ *   fa_fwd.
+ * Returns FA_OK once the kernels are queued.
+ */
+fa_status fa_fwd_keyrange(const void *q, const void *k, const void *v, void *o, fa_out_dtype o_dtype,
+                          float *lse, int B, int H, int Nq, int q_row0, int Nk, int k_pos0, int d,
+                          int causal, float scale, fa_stream_t stream);
+
+/*
+ * fa_merge_partials -- combine G attention partials of the same query rows over disjoint key
+ * ranges, with the rescaling rule of "Flash Attention" (myungum), section 2, steps 11-12, in
+ * log-sum-exp form: M = max_g LSE_g, w_g = exp(LSE_g - M), O = sum_g w_g O_g / sum_g w_g,
+ * LSE = M + ln sum_g w_g (a row whose partials are all -inf gets O = 0, LSE = -inf).
+ *
+ *   o_parts      fp32 [G, rows, d] contiguous, 16-byte aligned;  lse_parts: fp32 [G, rows].
+ *   o            [rows, d], bf16 or fp32 per o_dtype;  lse: fp32 [rows] or NULL.  Must not overlap
+ *                the partials.
+ *   G, rows >= 1;  d: 64 or 128.
+ * Returns FA_OK once the kernel is queued.
+ */
+fa_status fa_merge_partials(const float *o_parts, const float *lse_parts, int G, long long rows,
+                            int d, void *o, fa_out_dtype o_dtype, float *lse, fa_stream_t stream);
+
+/*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs: 4 * (d + 2) per query row, with
  * N rounded up to a multiple of 128.  Returns 0 on invalid sizes.
  */

@@ -132,6 +132,20 @@ def test_tree_attention_rejections(lib):
     assert tree(d=96) == 2
 
 
+def test_keyrange_and_merge_rejections(lib):
+    def kr(q_row0=0, Nk=64, k_pos0=0, Nq=100, d=128, o=7 * A, causal=0):
+        return lib.fa_fwd_keyrange(A, 2 * A, 3 * A, o, 1, 8 * A, 1, 2, Nq, q_row0, Nk, k_pos0, d,
+                                   causal, 0.0, None)
+    assert kr(q_row0=100) == 1 and kr(q_row0=-1) == 1 and kr(Nk=0) == 1 and kr(k_pos0=-5) == 1
+    assert kr(causal=2) == 1 and kr(d=32) == 2
+    assert kr(o=A + 64) == 1  # output overlaps q
+    def mg(G=2, rows=10, d=64, o=5 * A, parts=A):
+        return lib.fa_merge_partials(parts, 3 * A, G, rows, d, o, 0, None, None)
+    assert mg(G=0) == 1 and mg(rows=0) == 1 and mg(d=96) == 2
+    assert mg(parts=A + 4) == 3
+    assert mg(o=A + 128) == 1  # output overlaps the partials
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
