@@ -505,30 +505,70 @@ def bench_ours(args, rank, world):
         return result
 
     # ---- e2e through the Python API with host buffers: both launches of a step read the same
-    # Q, K, V (the two cases share one seed), so a step copies them to the device once, runs the
-    # non-causal and the causal forward, and copies both outputs (O and LSE) back.
+    # Q, K, V (the two cases share one seed), so a step copies them to the device once (pinned
+    # host -> device), runs the non-causal and the causal forward, and copies both outputs (O and
+    # LSE) back to pinned host memory.  Steps are pipelined over three streams with two device
+    # buffer sets: step t+1's inputs travel while step t computes and step t-1's outputs return
+    # (PCIe carries both directions at once).  The inputs (201 MB) exceed L2, so no flush is
+    # needed between steps; the time is the whole run's, divided by the step count.
     assert all(torch.equal(a, b) for a, b in zip(inputs[0], inputs[1]))
     host_in = [t.cpu().pin_memory() for t in inputs[0]]
     host_out = [(torch.empty(inputs[0][0].shape, dtype=torch.bfloat16).pin_memory(),
                  torch.empty(inputs[0][0].shape[:3], dtype=torch.float32).pin_memory()) for _ in cases]
-    dev_in = [torch.empty_like(t) for t in inputs[0]]
-    e2e_steps = max(3, min(args.steps, 20))
+    dev_in = [[torch.empty_like(t) for t in inputs[0]] for _ in range(2)]
+    dev_out = [[(torch.empty_like(inputs[0][0]),
+                 torch.empty(inputs[0][0].shape[:3], dtype=torch.float32, device=dev))
+                for _ in cases] for _ in range(2)]
+    del inputs, outs
+    torch.cuda.empty_cache()
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_comp + ev_out:
+        e.record(stream)
+    e2e_steps = max(4, min(args.steps, 20))
 
-    def e2e_step():
-        for h, d_ in zip(host_in, dev_in):
-            d_.copy_(h, non_blocking=True)
-        for c, (ho, hl) in zip(cases, host_out):
-            o, lse = fa.fa_fwd(dev_in[0], dev_in[1], dev_in[2], causal=c.causal, scale=c.scale)
-            ho.copy_(o, non_blocking=True)
-            hl.copy_(lse, non_blocking=True)
+    def e2e_run(n_steps):
+        for t in range(n_steps):
+            b = t % 2
+            s_in.wait_event(ev_comp[b])          # step t-2 has finished reading dev_in[b]
+            with torch.cuda.stream(s_in):
+                for h, d_ in zip(host_in, dev_in[b]):
+                    d_.copy_(h, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])         # step t-2's outputs have left dev_out[b]
+            q_, k_, v_ = dev_in[b]
+            for c, (o_, l_) in zip(cases, dev_out[b]):
+                fa.fa_fwd(q_, k_, v_, causal=c.causal, scale=c.scale, out=o_, lse=l_)
+            ev_comp[b].record(stream)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                for (ho, hl), (o_, l_) in zip(host_out, dev_out[b]):
+                    ho.copy_(o_, non_blocking=True)
+                    hl.copy_(l_, non_blocking=True)
+                ev_out[b].record(s_out)
 
-    e2e_ts = time_launches(e2e_step, e2e_steps, 2, flush, stream)
-    e2e_ms = dist_max(statistics.mean(e2e_ts))
+    e2e_run(2)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    e2e_run(e2e_steps)
+    s_out.wait_event(ev_comp[(e2e_steps - 1) % 2])
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    e2e_ms = dist_max(t0.elapsed_time(t1) / e2e_steps)
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during the e2e run")
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(o.numel() * o.element_size() + l.numel() * l.element_size() for o, l in host_out)
     e2e = {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
-    del inputs, outs, host_in, host_out, dev_in
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+           "pipelined": "3 streams, 2 device buffer sets: copy-in, compute and copy-out of "
+                        "consecutive steps overlap",
+           "gpu_launches_per_step": 2}
+    del host_in, host_out, dev_in, dev_out
     torch.cuda.empty_cache()
 
     # ---- sequence-length sweep (the pages' benchmark grid)

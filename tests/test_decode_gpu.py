@@ -85,3 +85,8 @@ def test_bad_block_id_is_reported_not_read():
     fa.fa_decode_paged(inp["q"], inp["k_pool"], inp["v_pool"], table, inp["seq_lens"])
     assert fa.device_status() == 1
     assert fa.device_status() == 0  # reading clears it
+
+
+def test_decode_long_context():
+    # one 131072-token context (8192 pages, 256 split chunks) beside short ones
+    run_decode(W.DecodeCase("long", S=3, H=4, d=128, lens=[131072, 5, 777]))

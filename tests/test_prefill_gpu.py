@@ -90,3 +90,15 @@ def test_repeatable_bitwise():
     o1, l1 = fa.fa_fwd(q, k, v, causal=True)
     o2, l2 = fa.fa_fwd(q, k, v, causal=True)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_long_sequence_128k(causal):
+    # one head pair over N = 131072 (1024 key blocks per row tile, 256 query-tile pairs per head):
+    # sampled rows, including the last ones, against the oracle
+    parity.run_prefill(W.PrefillCase("long_128k", 1, 2, 131072, 128, causal), torch.float32)
+
+
+def test_many_heads_short_rows():
+    # B*H = 4096 (b, h) slices of N = 129: many units, each a full tile plus a one-row tile
+    parity.run_prefill(W.PrefillCase("many_heads", 64, 64, 129, 64, True), torch.float32)
