@@ -49,9 +49,11 @@ struct BwdCfg {
   static constexpr int kXBytes = 128 * 128 * 2;
   static constexpr int kStages = 2;                // Q ring
   static constexpr int kDoStages = HD == 128 ? 1 : 2;  // dO ring (one stage frees room at d = 128)
-  // dQ staging: one 8 KB slot per read-out warp, boxes of 32 features x kBoxRows rows, fp32,
-  // 128-byte swizzle (d = 128: 64 query rows; d = 64: the warp's 32 query rows)
-  static constexpr int kBoxRows = HD == 128 ? 64 : 32;
+  // dQ staging: one 8 KB slot per read-out warp, boxes of 32 features x 32 rows (4 KB), fp32,
+  // 128-byte swizzle.  d = 128: the slot's two halves take the warp's boxes in turn (one is
+  // written while the other is read by its reduction; 32-row boxes measured faster than 64, 16 or
+  // 8); d = 64: the warp's two boxes of its 32 query rows.
+  static constexpr int kBoxRows = 32;
   static constexpr int kStageSlotBytes = 8192;
   static constexpr int kVecFloats = 2 * kBM;       // LSE (log2 units) and D of one query block
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + HD;
@@ -167,29 +169,36 @@ __device__ __forceinline__ void read_out_dq(uint32_t tq, int w, int lane, uint8_
                                             const CUtensorMap *tm_dq, int row0, uint64_t *dq_free) {
   using C = BwdCfg<HD>;
   if constexpr (C::kDqT) {
+    // boxes of kBoxRows query rows, cycling through the slot's kBufs buffers: a box is written
+    // while the kBufs - 1 before it are still being read by their reductions
+    constexpr int kRows = C::kBoxRows, kBufs = C::kStageSlotBytes / (kRows * 128);
 #pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-      uint32_t v[2][32];
-      tmem_ld32(tq + 64 * half, v[0]);
-      tmem_ld32(tq + 64 * half + 32, v[1]);
+    for (int q0 = 0; q0 < kBM; q0 += 32) {
+      uint32_t v[32];
+      tmem_ld32(tq + q0, v);
       tmem_wait_ld();
-      if (half == 1) {  // TMEM fully read: the columns may take the next block's S^T
+      if (q0 + 32 == kBM) {  // TMEM fully read: the columns may take the next block's S^T
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_free);
       }
-      if (lane == 0) bulk_wait_group_read<0>();  // the previous box has left the slot
-      __syncwarp();
-      const int unit = lane / 4, sub = (lane % 4) * 4;
 #pragma unroll
-      for (int q = 0; q < 64; ++q)
-        *reinterpret_cast<float *>(slot + q * 128 + ((unit ^ (q & 7)) * 16) + sub) =
-            __uint_as_float(v[q / 32][q % 32]);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_reduce_add_2d(tm_dq, slot, 32 * w, row0 + 64 * half);
-        bulk_commit_group();
+      for (int b0 = 0; b0 < 32; b0 += kRows) {
+        const int bi = (q0 + b0) / kRows;
+        if (lane == 0) bulk_wait_group_read<kBufs - 1>();  // this buffer's last box has left it
+        __syncwarp();
+        uint8_t *box = slot + (bi % kBufs) * (kRows * 128);
+        const int unit = lane / 4, sub = (lane % 4) * 4;
+#pragma unroll
+        for (int q = 0; q < kRows; ++q)
+          *reinterpret_cast<float *>(box + q * 128 + ((unit ^ (q & 7)) * 16) + sub) =
+              __uint_as_float(v[b0 + q]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_2d(tm_dq, box, 32 * w, row0 + q0 + b0);
+          bulk_commit_group();
+        }
       }
     }
   } else {
