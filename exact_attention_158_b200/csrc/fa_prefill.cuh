@@ -59,8 +59,10 @@ struct PrefillCfg {
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + HD;
   static constexpr uint32_t kColP0 = 256 + 2 * HD, kColP1 = kColP0 + kBN / 2;  // TMEM P (d = 64)
   static constexpr int kNumBars = 2 + 2 * kStages + 4 * 2 + 1;
+  static constexpr int kSchedBytes = 2 * 128 * 4;  // paged mode: sequence lengths and their order
   static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + 2 * kTileBytes +
-                                       kStages * kTileBytes + 2 * kPBytes + kNumBars * 8 + 16;
+                                       kStages * kTileBytes + 2 * kPBytes + kNumBars * 8 + 16 +
+                                       kSchedBytes;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, 0, 1);   // P K-major, V MN-major
@@ -127,22 +129,35 @@ struct WorkUnit {
   int pair;
 };
 
+// Paged units cost in proportion to their sequence's cached length, which only the device
+// knows.  With at most kMaxSortedSeqs sequences each CTA ranks them itself at start-up (longest
+// first, ties by index; the same order in every CTA) and numbers the units sequence by sequence in
+// that order, dealt in snake order like the causal levels; with more sequences, or in the
+// key-range mode, units are numbered head-major and dealt round-robin.
+constexpr int kMaxSortedSeqs = 128;
+
 // The unit CTA blockIdx.x processes in its round r, or -1 once it has none left.
-// (Paged and key-range units are numbered head-major like non-causal ones: their costs depend on
-// per-unit spans that the longest-first order does not model.)
-template <bool kPaged = false>
-__device__ __forceinline__ int unit_for_round(const PrefillParams &p, int r) {
+template <bool kGeneral = false>
+__device__ __forceinline__ int unit_for_round(const PrefillParams &p, int r,
+                                              const int *seq_order = nullptr) {
   const int G = gridDim.x, c = blockIdx.x;
-  const int u = r * G + ((!kPaged && p.causal && (r & 1)) ? G - 1 - c : c);
+  const bool snake = kGeneral ? seq_order != nullptr : p.causal;
+  const int u = r * G + ((snake && (r & 1)) ? G - 1 - c : c);
   return u < p.num_units ? u : -1;
 }
 
-template <bool kPaged = false>
-__device__ __forceinline__ WorkUnit decode_unit(const PrefillParams &p, int u) {
+template <bool kGeneral = false>
+__device__ __forceinline__ WorkUnit decode_unit(const PrefillParams &p, int u,
+                                                const int *seq_order = nullptr) {
   WorkUnit w;
-  if (!kPaged && p.causal) {
+  if (!kGeneral && p.causal) {
     w.bh = u % p.BH;
     w.pair = p.num_pairs - 1 - u / p.BH;
+  } else if (kGeneral && seq_order != nullptr) {
+    const int per_seq = p.H * p.num_pairs;
+    const int rem = u % per_seq;
+    w.bh = seq_order[u / per_seq] * p.H + rem / p.num_pairs;
+    w.pair = rem % p.num_pairs;
   } else {
     w.bh = u / p.num_pairs;
     w.pair = u % p.num_pairs;
@@ -300,9 +315,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t *drain = pv_done + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *s_lens = const_cast<int *>(reinterpret_cast<volatile int *>(abort_flag + 1));  // [128]
+  int *s_order = s_lens + kMaxSortedSeqs;                                              // [128]
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  // paged mode with few sequences: longest-first order of the sequences (computed below)
+  const int n_seqs = kPaged ? p.BH / p.H : 0;
+  const int *seq_order = (kPaged && n_seqs <= kMaxSortedSeqs) ? s_order : nullptr;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -329,6 +349,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+  }
+  if (seq_order != nullptr && warp == 10) {
+    // rank the sequences by cached length (clamped as the units will see it), longest first
+    for (int sq = lane; sq < n_seqs; sq += 32) s_lens[sq] = kv_span<kMode>(p, sq * p.H).L;
+    __syncwarp();
+    for (int sq = lane; sq < n_seqs; sq += 32) {
+      const int L = s_lens[sq];
+      int rank = 0;
+      for (int o = 0; o < n_seqs; ++o) {
+        const int Lo = s_lens[o];
+        rank += (Lo > L || (Lo == L && o < sq)) ? 1 : 0;
+      }
+      s_order[rank] = sq;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -384,9 +418,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         return true;
       };
       for (int r = 0; ok; ++r) {
-        const int u = unit_for_round<kGeneral>(p, r);
+        const int u = unit_for_round<kGeneral>(p, r, seq_order);
         if (u < 0) break;
-        const WorkUnit w = decode_unit<kGeneral>(p, u);
+        const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
         const int pr = w.pair;
         const KvSpan kv = kv_span<kMode>(p, w.bh);
         kv_len = kv.L;
@@ -437,9 +471,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
         bool ok = true;
         for (int r = 0; ok; ++r) {
-          const int u = unit_for_round<kGeneral>(p, r);
+          const int u = unit_for_round<kGeneral>(p, r, seq_order);
           if (u < 0) break;
-          const WorkUnit w = decode_unit<kGeneral>(p, u);
+          const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
           const int pr = w.pair;
           const KvSpan kv = kv_span<kMode>(p, w.bh);
           const int n[2] = {tile_blocks(p, kv, pr, 0), tile_blocks(p, kv, pr, 1)};
@@ -535,9 +569,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           return true;
         };
         for (int r = 0; ok; ++r) {
-          const int u = unit_for_round<kGeneral>(p, r);
+          const int u = unit_for_round<kGeneral>(p, r, seq_order);
           if (u < 0) break;
-          const WorkUnit w = decode_unit<kGeneral>(p, u);
+          const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
           const int pr = w.pair;
           const KvSpan kv = kv_span<kMode>(p, w.bh);
           const int n[2] = {tile_blocks(p, kv, pr, 0), tile_blocks(p, kv, pr, 1)};
@@ -603,9 +637,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t s_ph = 0, pv_ph = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-      const int u = unit_for_round<kGeneral>(p, r);
+      const int u = unit_for_round<kGeneral>(p, r, seq_order);
       if (u < 0) break;
-      const WorkUnit w = decode_unit<kGeneral>(p, u);
+      const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
       const int pr = w.pair;
       const KvSpan kv = kv_span<kMode>(p, w.bh);
       const int n = tile_blocks(p, kv, pr, wg);
