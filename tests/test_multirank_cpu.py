@@ -33,7 +33,7 @@ def _worker(rank, world, port, out):
 
 def test_aggregate_takes_the_slowest_rank():
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
     for rank in range(2):

@@ -54,7 +54,7 @@ def _worker(rank, world, port, causal, out):
 @pytest.mark.parametrize("causal", [False, True])
 def test_sharded_keys_merge_to_plain_attention(world, causal):
     port = _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, port, causal, out), nprocs=world, join=True)
     for rank in range(world):
         do, dl = out[rank]
