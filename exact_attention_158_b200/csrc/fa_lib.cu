@@ -560,7 +560,8 @@ static fa_status prefill_paged_impl(const void *q, const void *k_pool, const voi
   if (overlaps(o, o_bytes, q, q_bytes) || overlaps(o, o_bytes, k_pool, pool_bytes) ||
       overlaps(o, o_bytes, v_pool, pool_bytes))
     return FA_ERR_INVALID_ARG;
-  if (lse && (overlaps(lse, rows * 4, o, o_bytes) || overlaps(lse, rows * 4, q, q_bytes)))
+  if (lse && (overlaps(lse, rows * 4, o, o_bytes) || overlaps(lse, rows * 4, q, q_bytes) ||
+              overlaps(lse, rows * 4, k_pool, pool_bytes) || overlaps(lse, rows * 4, v_pool, pool_bytes)))
     return FA_ERR_INVALID_ARG;
   DeviceInfo *dev = nullptr;
   int dev_id = 0;
@@ -640,7 +641,8 @@ fa_status fa_fwd_keyrange(const void *q, const void *k, const void *v, void *o, 
   if (overlaps(o, o_bytes, q, qrows * d * 2) || overlaps(o, o_bytes, k, krows * d * 2) ||
       overlaps(o, o_bytes, v, krows * d * 2))
     return FA_ERR_INVALID_ARG;
-  if (lse && (overlaps(lse, qrows * 4, o, o_bytes) || overlaps(lse, qrows * 4, q, qrows * d * 2)))
+  if (lse && (overlaps(lse, qrows * 4, o, o_bytes) || overlaps(lse, qrows * 4, q, qrows * d * 2) ||
+              overlaps(lse, qrows * 4, k, krows * d * 2) || overlaps(lse, qrows * 4, v, krows * d * 2)))
     return FA_ERR_INVALID_ARG;
   DeviceInfo *dev = nullptr;
   int dev_id = 0;

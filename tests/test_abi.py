@@ -139,6 +139,8 @@ def test_keyrange_and_merge_rejections(lib):
     assert kr(q_row0=100) == 1 and kr(q_row0=-1) == 1 and kr(Nk=0) == 1 and kr(k_pos0=-5) == 1
     assert kr(causal=2) == 1 and kr(d=32) == 2
     assert kr(o=A + 64) == 1  # output overlaps q
+    assert lib.fa_fwd_keyrange(A, 2 * A, 3 * A, 7 * A, 1, 2 * A + 64, 1, 2, 100, 0, 64, 0, 128, 0,
+                               0.0, None) == 1  # LSE overlaps k
     def mg(G=2, rows=10, d=64, o=5 * A, parts=A):
         return lib.fa_merge_partials(parts, 3 * A, G, rows, d, o, 0, None, None)
     assert mg(G=0) == 1 and mg(rows=0) == 1 and mg(d=96) == 2
