@@ -8,9 +8,11 @@
  * Q, K, V are loaded into on-chip memory, the row max m and row sum l are carried across key
  * blocks, and only O, l, m are written back; "How Flash Attention reduces memory traffic"
  * (zimaspace), tiling and online softmax).  Work is split over batch, head and query tile
- * ("FlashAttention-2 GPU work partitioning", section 3).  The paged decode entry point reads its
- * keys and values through a block table that maps each sequence's logical KV blocks to physical
- * blocks of a shared pool ("LLM study notes" (devocean.sk.com), paged attention).
+ * ("FlashAttention-2 GPU work partitioning", section 3).  The paged entry points (decode, chunked
+ * prefill, draft-tree verification) read keys and values through a block table that maps each
+ * sequence's logical KV blocks to physical blocks of a shared pool ("LLM study notes"
+ * (devocean.sk.com), paged attention).  Key-range partials and their merge serve a sequence whose
+ * keys are split across devices.
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never allocates,
@@ -42,12 +44,12 @@ typedef enum {
     FA_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned                                  */
     FA_ERR_LAUNCH = 4,      /* the CUDA launch failed; fa_last_error_string() has the CUDA text  */
     FA_ERR_TIMEOUT = 5,     /* a kernel gave up waiting (reported by fa_get_device_status)       */
-    FA_ERR_WORKSPACE = 6    /* the decode workspace is NULL or smaller than required             */
+    FA_ERR_WORKSPACE = 6    /* a workspace is NULL or smaller than required (decode, backward)   */
 } fa_status;
 
 typedef enum {
-    FA_OUT_BF16 = 0, /* O written as bf16 (round to nearest even) */
-    FA_OUT_F32 = 1   /* O written as fp32                          */
+    FA_OUT_BF16 = 0, /* written as bf16 (round to nearest even) */
+    FA_OUT_F32 = 1   /* written as fp32                          */
 } fa_out_dtype;
 
 /*
