@@ -93,15 +93,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [BH, N, d] bf16 viewed as a 3-D tensor (d innermost); boxes of 64 x 128 x 1 with 128-byte
-// swizzle, rows past N read as zeros.
-bool encode_bhnd(CUtensorMap *map, const void *base, int d, int N, int BH) {
+// [BH, N, d] bf16 viewed as a 3-D tensor (d innermost); boxes of 64 x box_rows x 1 with 128-byte
+// swizzle, rows past N read as zeros (and not written by stores).
+bool encode_bhnd(CUtensorMap *map, const void *base, int d, int N, int BH, int box_rows = 128) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -156,7 +156,8 @@ bool encode_pool(CUtensorMap *map, const void *base, int d, int H, int num_block
 
 template <int HD, int kMode>
 fa_status launch_prefill(DeviceInfo &dev, const CUtensorMap &tq, const CUtensorMap &tk,
-                         const CUtensorMap &tv, fa::PrefillParams p, cudaStream_t stream) {
+                         const CUtensorMap &tv, fa::PrefillParams p, cudaStream_t stream,
+                         const CUtensorMap *to = nullptr) {
   using C = fa::PrefillCfg<HD>;
   p.num_pairs = (p.N + 2 * fa::kBM - 1) / (2 * fa::kBM);
   p.num_units = p.BH * p.num_pairs;
@@ -172,8 +173,9 @@ fa_status launch_prefill(DeviceInfo &dev, const CUtensorMap &tq, const CUtensorM
     }
   }
   const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
-  fa::fa_prefill_kernel<HD, kMode><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk,
-                                                                                         tv, p);
+  // without an O map (p.o_tma = 0) the kernel never reads its O map argument
+  fa::fa_prefill_kernel<HD, kMode><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(
+      tq, tk, tv, to != nullptr ? *to : tq, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : launch_failed(e);
 }
@@ -198,7 +200,10 @@ fa_status launch_prefill_dense(DeviceInfo &dev, const void *q, const void *k, co
   p.scale_log2 = scale * 1.4426950408889634f;
   p.q_rows = N;
   p.Nk = N;
-  return launch_prefill<HD, fa::kModeSquare>(dev, tq, tk, tv, p, stream);
+  // bf16 O at d = 128 leaves through tensor stores of 32-row boxes
+  CUtensorMap to;
+  p.o_tma = (HD == 128 && !o_f32 && encode_bhnd(&to, o, HD, N, BH, 32)) ? 1 : 0;
+  return launch_prefill<HD, fa::kModeSquare>(dev, tq, tk, tv, p, stream, p.o_tma ? &to : nullptr);
 }
 
 // Backward workspace: dQ accumulator fp32 [BH, Np, d], then LSE2 and D fp32 [BH, Np] each, with

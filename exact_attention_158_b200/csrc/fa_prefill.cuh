@@ -28,6 +28,17 @@
 
 namespace fa {
 
+// Tile store shared -> global through a 3-D tensor map (rows past the map's extent are not
+// written); completion is tracked by this thread's bulk groups.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per key/value block
 constexpr int kPrefillThreads = 384;
@@ -90,6 +101,9 @@ struct PrefillParams {
   // with q_rows rows per (b, h); the keys are the Nk rows of K / V; query row r sits at key
   // position q_off + r (>= 0).  The other modes use q_row0 = 0 and q_rows = N.
   int q_row0, q_rows, Nk, q_off;
+  // square mode, d = 128, bf16 O: 1 when the O tensor map was encoded, so the epilogue stages O in
+  // the tile's (by then unused) P buffer and writes it with tensor stores
+  int o_tma;
 };
 
 // Kernel modes: square prefill (keys = queries), paged cache (keys gathered through the block
@@ -293,10 +307,13 @@ template <int HD, int kMode>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
   using C = PrefillCfg<HD>;
   constexpr bool kPaged = kMode == kModePaged;
   constexpr bool kGeneral = kMode != kModeSquare;  // key count and query offset per unit
+  // O through the P tile and tensor stores (square mode with P in shared memory; bf16 O)
+  constexpr bool kTmaO = !kGeneral && !C::kPInTmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -349,6 +366,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    if (kTmaO && p.o_tma) tma_prefetch_desc(&tm_o);
   }
   if (seq_order != nullptr && warp == 10) {
     // rank the sequences by cached length (clamped as the units will see it), longest first
@@ -728,6 +746,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_st32(tP, pk);
           tmem_st32(tP + 32, pk + 32);
         } else {
+          if (kTmaO && p.o_tma && j == 0) {
+            // the previous unit's O left this warp's rows of the P tile through tensor stores
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+          }
           store_p_row(pTile, row, pk);
         }
         if (j > 0) {
@@ -763,6 +786,38 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const bool live = qrow < p.N;
       const size_t grow = kGeneral ? static_cast<size_t>(w.bh) * p.q_rows + p.q_row0 + qrow
                                    : static_cast<size_t>(w.bh) * p.N + qrow;
+      if (kTmaO && p.o_tma) {
+        // O / l as bf16 into this thread's row of the P tile (the layout P uses: 64 columns per
+        // 128-byte-swizzled chunk), then one tensor store per chunk of the warp's 32 rows
+#pragma unroll
+        for (int cc = 0; cc < HD; cc += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc, o);
+          tmem_wait_ld();
+          uint8_t *rowp = pTile + (cc / 64) * C::kChunkBytes + row * 128;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int u = (cc % 64) / 8 + e;
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
+            *reinterpret_cast<uint4 *>(rowp + ((u ^ (row & 7)) * 16)) = v;
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        const int r0 = qrow - lane;  // the warp's first row; boxes reaching past N are clipped
+        if (lane == 0 && r0 < p.N) {
+#pragma unroll
+          for (int ch = 0; ch < HD / 64; ++ch)
+            tma_store_3d(&tm_o, pTile + ch * C::kChunkBytes + (row - lane) * 128, 64 * ch, r0, w.bh);
+          bulk_commit_group();
+        }
+        if (live && p.lse) p.lse[grow] = (m_ref + lg2(l)) * kLn2;
+        continue;
+      }
 #pragma unroll
       for (int cc = 0; cc < HD; cc += 32) {
         uint32_t o[32];
@@ -790,6 +845,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
       if (live && p.lse) p.lse[grow] = (m_ref + lg2(l)) * kLn2;
+    }
+    if (kTmaO && p.o_tma) {
+      if (lane == 0) bulk_wait_group_all();  // the stores have read the P tile before the CTA exits
+      __syncwarp();
     }
   }
 

@@ -22,6 +22,15 @@ def test_ragged_lengths(N, causal, d):
     parity.run_prefill(W.PrefillCase(f"ragged_N{N}", 2, 2, N, d, causal), torch.float32, full=True)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 31, 32, 33, 129, 255, 1000])
+def test_ragged_lengths_bf16_out(N, causal, d):
+    # bf16 O: at d = 128 it leaves through tensor stores of 32-row boxes, clipped at row N
+    parity.run_prefill(W.PrefillCase(f"ragged_bf16_N{N}", 2, 3, N, d, causal), torch.bfloat16,
+                       full=True)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_multi_tile_full(causal):
     # several heads, 8 query pairs, 16 key blocks: exercises the ring, the persistent loop and
@@ -81,6 +90,23 @@ def test_guard_bytes_untouched():
     assert torch.isnan(buf[:pad]).all() and torch.isnan(buf[pad + n:]).all()
     assert torch.isnan(lbuf[:pad]).all() and torch.isnan(lbuf[pad + 600:]).all()
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_guard_bytes_untouched_bf16_out(d):
+    # bf16 O written into the middle of a NaN-filled buffer: nothing outside [B, H, N, d] changes,
+    # also where the last 32-row box of a head reaches past N
+    import exact_attention_158_b200 as fa
+    case = W.PrefillCase("guard_bf16", 1, 3, 200, d, False)
+    q, k, v = W.make_prefill(case, device="cuda")
+    n = 3 * 200 * d
+    pad = 4096
+    buf = torch.full((n + 2 * pad,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    o = buf[pad:pad + n].view(1, 3, 200, d)
+    fa.fa_fwd(q, k, v, causal=False, out_dtype=torch.bfloat16, out=o)
+    torch.cuda.synchronize()
+    assert torch.isnan(buf[:pad]).all() and torch.isnan(buf[pad + n:]).all()
+    assert torch.isfinite(o).all()
 
 
 def test_repeatable_bitwise():
