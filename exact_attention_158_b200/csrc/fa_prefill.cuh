@@ -23,6 +23,9 @@
 // the MMA warp then computes S_i,j+1 while the softmax is still turning S_i,j into P_i,j, and
 // O_i += P_i,j V_j follows when P_i,j is ready.  Each softmax warpgroup thus runs back to back,
 // and the two tiles keep the tensor core fed in turn.
+// Epilogue: O_i / l_i per row.  In the square mode with bf16 O at d = 128 each warp stages its 32
+// rows in the (then unused) P buffer and writes them with TMA tensor stores, so the warp starts the
+// next unit while the stores drain; otherwise every thread stores its own row.
 #pragma once
 #include "sm100_ptx.cuh"
 
