@@ -200,9 +200,9 @@ fa_status launch_prefill_dense(DeviceInfo &dev, const void *q, const void *k, co
   p.scale_log2 = scale * 1.4426950408889634f;
   p.q_rows = N;
   p.Nk = N;
-  // bf16 O at d = 128 leaves through tensor stores of 32-row boxes
+  // bf16 O leaves through tensor stores of 32-row boxes
   CUtensorMap to;
-  p.o_tma = (HD == 128 && !o_f32 && encode_bhnd(&to, o, HD, N, BH, 32)) ? 1 : 0;
+  p.o_tma = (!o_f32 && encode_bhnd(&to, o, HD, N, BH, 32)) ? 1 : 0;
   return launch_prefill<HD, fa::kModeSquare>(dev, tq, tk, tv, p, stream, p.o_tma ? &to : nullptr);
 }
 

@@ -23,9 +23,10 @@
 // the MMA warp then computes S_i,j+1 while the softmax is still turning S_i,j into P_i,j, and
 // O_i += P_i,j V_j follows when P_i,j is ready.  Each softmax warpgroup thus runs back to back,
 // and the two tiles keep the tensor core fed in turn.
-// Epilogue: O_i / l_i per row.  In the square mode with bf16 O at d = 128 each warp stages its 32
-// rows in the (then unused) P buffer and writes them with TMA tensor stores, so the warp starts the
-// next unit while the stores drain; otherwise every thread stores its own row.
+// Epilogue: O_i / l_i per row.  In the square mode with bf16 O each warp stages its 32 rows in
+// shared memory (d = 128: the then unused P buffer; d = 64: a staging tile of its own) and writes
+// them with TMA tensor stores, so the warp starts the next unit while the stores drain; otherwise
+// every thread stores its own row.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -66,6 +67,9 @@ struct PrefillCfg {
   // faster; at d = 128 the fixed order S_0,j+1  S_1,j+1  PV_0,j  PV_1,j did.
   static constexpr bool kEventMma = HD == 64;
   static constexpr int kPBytes = kPInTmem ? 0 : 128 * kBN * 2;  // one 128 x 128 bf16 P tile
+  // bf16 O staging for the tensor-store epilogue: the P tile where there is one, else a buffer of
+  // its own per query tile (d = 64: 128 rows x 128 bytes)
+  static constexpr int kOStageBytes = kPInTmem ? 128 * HD * 2 : 0;
   // K/V ring depth: K_{j+1} is loaded one block ahead of V_j, so three stages give every load
   // about one block of slack.
   static constexpr int kStages = HD == 128 ? 3 : 8;
@@ -75,8 +79,8 @@ struct PrefillCfg {
   static constexpr int kNumBars = 2 + 2 * kStages + 4 * 2 + 1;
   static constexpr int kSchedBytes = 2 * 128 * 4;  // paged mode: sequence lengths and their order
   static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + 2 * kTileBytes +
-                                       kStages * kTileBytes + 2 * kPBytes + kNumBars * 8 + 16 +
-                                       kSchedBytes;
+                                       kStages * kTileBytes + 2 * kPBytes + 2 * kOStageBytes +
+                                       kNumBars * 8 + 16 + kSchedBytes;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, 0, 1);   // P K-major, V MN-major
@@ -315,15 +319,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   using C = PrefillCfg<HD>;
   constexpr bool kPaged = kMode == kModePaged;
   constexpr bool kGeneral = kMode != kModeSquare;  // key count and query offset per unit
-  // O through the P tile and tensor stores (square mode with P in shared memory; bf16 O)
-  constexpr bool kTmaO = !kGeneral && !C::kPInTmem;
+  // bf16 O through a shared-memory staging tile and tensor stores (square mode)
+  constexpr bool kTmaO = !kGeneral;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sQ = smem;                                   // 2 tiles
   uint8_t *sKV = sQ + 2 * C::kTileBytes;                // kStages tiles
   uint8_t *sP = sKV + C::kStages * C::kTileBytes;       // 2 P tiles
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sP + 2 * C::kPBytes);
+  uint8_t *sO = sP + 2 * C::kPBytes;                     // 2 O staging tiles (d = 64)
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sO + 2 * C::kOStageBytes);
   uint64_t *q_full = bars;
   uint64_t *q_empty = bars + 1;
   uint64_t *kv_full = bars + 2;
@@ -653,6 +658,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t tS = tmem + lane_off + (wg ? C::kColS1 : C::kColS0);
     const uint32_t tO = tmem + lane_off + (wg ? C::kColO1 : C::kColO0);
     uint8_t *pTile = sP + wg * C::kPBytes;
+    uint8_t *oTile = C::kPInTmem ? sO + wg * C::kOStageBytes : pTile;
     const uint32_t tP = tmem + lane_off + (wg ? C::kColP1 : C::kColP0);
     const float sl2 = p.scale_log2;
     uint32_t s_ph = 0, pv_ph = 0;
@@ -749,7 +755,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_st32(tP, pk);
           tmem_st32(tP + 32, pk + 32);
         } else {
-          if (kTmaO && p.o_tma && j == 0) {
+          if (kTmaO && !C::kPInTmem && p.o_tma && j == 0) {
             // the previous unit's O left this warp's rows of the P tile through tensor stores
             if (lane == 0) bulk_wait_group_read<0>();
             __syncwarp();
@@ -790,14 +796,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const size_t grow = kGeneral ? static_cast<size_t>(w.bh) * p.q_rows + p.q_row0 + qrow
                                    : static_cast<size_t>(w.bh) * p.N + qrow;
       if (kTmaO && p.o_tma) {
-        // O / l as bf16 into this thread's row of the P tile (the layout P uses: 64 columns per
-        // 128-byte-swizzled chunk), then one tensor store per chunk of the warp's 32 rows
+        // O / l as bf16 into this thread's row of the staging tile (the layout P uses: 64 columns
+        // per 128-byte-swizzled chunk), then one tensor store per chunk of the warp's 32 rows.  A
+        // staging tile of its own (d = 64) still holds this warp's rows of the previous unit's O
+        // until those stores have read it.
+        if constexpr (C::kPInTmem) {
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+        }
 #pragma unroll
         for (int cc = 0; cc < HD; cc += 32) {
           uint32_t o[32];
           tmem_ld32(tO + cc, o);
           tmem_wait_ld();
-          uint8_t *rowp = pTile + (cc / 64) * C::kChunkBytes + row * 128;
+          uint8_t *rowp = oTile + (cc / 64) * C::kChunkBytes + row * 128;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int u = (cc % 64) / 8 + e;
@@ -815,7 +827,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (lane == 0 && r0 < p.N) {
 #pragma unroll
           for (int ch = 0; ch < HD / 64; ++ch)
-            tma_store_3d(&tm_o, pTile + ch * C::kChunkBytes + (row - lane) * 128, 64 * ch, r0, w.bh);
+            tma_store_3d(&tm_o, oTile + ch * C::kChunkBytes + (row - lane) * 128, 64 * ch, r0, w.bh);
           bulk_commit_group();
         }
         if (live && p.lse) p.lse[grow] = (m_ref + lg2(l)) * kLn2;
