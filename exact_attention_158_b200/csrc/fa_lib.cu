@@ -595,8 +595,12 @@ static fa_status prefill_paged_impl(const void *q, const void *k_pool, const voi
   p.tree_mask = tree_mask;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   p.q_rows = Lq;
-  if (d == 128) return launch_prefill<128, fa::kModePaged>(*dev, tq, tk, tv, p, s);
-  return launch_prefill<64, fa::kModePaged>(*dev, tq, tk, tv, p, s);
+  // bf16 O leaves through tensor stores of 32-row boxes ([S * H, Lq, d] view)
+  CUtensorMap to;
+  p.o_tma = (o_dtype == FA_OUT_BF16 && encode_bhnd(&to, o, d, Lq, BH, 32)) ? 1 : 0;
+  const CUtensorMap *top = p.o_tma ? &to : nullptr;
+  if (d == 128) return launch_prefill<128, fa::kModePaged>(*dev, tq, tk, tv, p, s, top);
+  return launch_prefill<64, fa::kModePaged>(*dev, tq, tk, tv, p, s, top);
 }
 
 fa_status fa_prefill_paged(const void *q, const void *k_pool, const void *v_pool,

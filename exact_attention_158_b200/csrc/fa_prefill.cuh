@@ -23,10 +23,10 @@
 // the MMA warp then computes S_i,j+1 while the softmax is still turning S_i,j into P_i,j, and
 // O_i += P_i,j V_j follows when P_i,j is ready.  Each softmax warpgroup thus runs back to back,
 // and the two tiles keep the tensor core fed in turn.
-// Epilogue: O_i / l_i per row.  In the square mode with bf16 O each warp stages its 32 rows in
-// shared memory (d = 128: the then unused P buffer; d = 64: a staging tile of its own) and writes
-// them with TMA tensor stores, so the warp starts the next unit while the stores drain; otherwise
-// every thread stores its own row.
+// Epilogue: O_i / l_i per row.  In the square and paged modes with bf16 O each warp stages its
+// 32 rows in shared memory (d = 128: the then unused P buffer; d = 64: a staging tile of its own)
+// and writes them with TMA tensor stores, so the warp starts the next unit while the stores drain;
+// otherwise every thread stores its own row.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -319,8 +319,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   using C = PrefillCfg<HD>;
   constexpr bool kPaged = kMode == kModePaged;
   constexpr bool kGeneral = kMode != kModeSquare;  // key count and query offset per unit
-  // bf16 O through a shared-memory staging tile and tensor stores (square mode)
-  constexpr bool kTmaO = !kGeneral;
+  // bf16 O through a shared-memory staging tile and tensor stores (square and paged modes: the
+  // processed rows of (b, h) are rows 0 .. N-1 of its O slice)
+  constexpr bool kTmaO = kMode != kModeRange;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

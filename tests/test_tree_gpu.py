@@ -45,8 +45,9 @@ def test_tree_shapes(shape):
     parity.assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, f"tree {shape}")
 
 
-def test_tree_bf16_out():
-    case = W.DecodeCase("tree_bf16", S=4, H=4, d=128, lens=[96, 300, 1000, 50])
+@pytest.mark.parametrize("d", [64, 128])
+def test_tree_bf16_out(d):
+    case = W.DecodeCase(f"tree_bf16_d{d}", S=4, H=4, d=d, lens=[96, 300, 1000, 50])
     _, o, lse, o_ref, lse_ref = run_tree(case, 40, out_dtype=torch.bfloat16)
     parity.assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "tree bf16",
                         out_bf16=True)
