@@ -82,6 +82,7 @@ struct BwdParams {
   float *dq_acc;      // [BH, Np, d] fp32, zero before the launch
   void *dk, *dv;      // [BH, N, d]
   int g_f32;          // dK / dV as fp32 (1) or bf16 (0)
+  int g_tma;          // d = 128, bf16 dK / dV: written by tensor stores (their maps were encoded)
   int BH, N, Np, nkb, causal;
   float scale_log2, scale;
 };
@@ -151,6 +152,28 @@ __device__ __forceinline__ void store_grad_cols(uint32_t taddr, int c0, float mu
         w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
         dst[e] = w;
       }
+    }
+  }
+}
+
+// d = 128, bf16 gradients: this thread's row (64 features from column c0 of TMEM, times mul) as
+// bf16 into row `lane` of a 32-row x 128-byte box, 128-byte swizzle (16-byte unit u at u ^ (r % 8)).
+__device__ __forceinline__ void stage_grad_box(uint32_t taddr, int c0, float mul, uint8_t *box,
+                                               int lane) {
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    uint32_t v[32];
+    tmem_ld32(taddr + c0 + 32 * ch, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint4 w;
+      w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * mul, __uint_as_float(v[8 * e + 1]) * mul);
+      w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * mul, __uint_as_float(v[8 * e + 3]) * mul);
+      w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * mul, __uint_as_float(v[8 * e + 5]) * mul);
+      w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
+      const int u = ch * 4 + e;
+      *reinterpret_cast<uint4 *>(box + lane * 128 + ((u ^ (lane & 7)) * 16)) = w;
     }
   }
 }
@@ -233,7 +256,9 @@ template <int HD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq,
+                  const __grid_constant__ CUtensorMap tm_dk,
+                  const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using C = BwdCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
@@ -526,11 +551,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // dV_j and dK_j (times scale) once every MMA has completed
     if (ok && __all_sync(0xffffffffu, mbar_wait(dq_full, (n - 1) & 1, abort_flag))) {
       tc_fence_after();
-      const size_t grow = static_cast<size_t>(bh) * p.N + jb * kBN + r;
-      store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDV, h * (HD / 2), 1.f, p.dv, p.g_f32,
-                                   grow, key_live);
-      store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDK, h * (HD / 2), p.scale, p.dk,
-                                   p.g_f32, grow, key_live);
+      if (HD == 128 && p.g_tma) {
+        // each warp's 32 key rows x 64 features of dV and dK: staged in the Q ring (every MMA
+        // that read it has completed) and written with one tensor store each, clipped at row N
+        uint8_t *box_v = sQ + warp * 4096, *box_k = sQ + 8 * 4096 + warp * 4096;
+        stage_grad_box(tmem + lane_off + C::kColDV, h * 64, 1.f, box_v, lane);
+        stage_grad_box(tmem + lane_off + C::kColDK, h * 64, p.scale, box_k, lane);
+        fence_async_smem();
+        __syncwarp();
+        const int r0 = jb * kBN + 32 * w4;
+        if (lane == 0 && r0 < p.N) {
+          tma_store_3d(&tm_dv, box_v, 64 * h, r0, bh);
+          tma_store_3d(&tm_dk, box_k, 64 * h, r0, bh);
+          bulk_commit_group();
+          bulk_wait_group_all();  // the boxes have been read before the CTA retires
+        }
+        __syncwarp();
+      } else {
+        const size_t grow = static_cast<size_t>(bh) * p.N + jb * kBN + r;
+        store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDV, h * (HD / 2), 1.f, p.dv,
+                                     p.g_f32, grow, key_live);
+        store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDK, h * (HD / 2), p.scale, p.dk,
+                                     p.g_f32, grow, key_live);
+      }
     }
   }
 

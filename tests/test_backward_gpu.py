@@ -33,6 +33,14 @@ def test_backward_bf16_grads(d):
     parity.run_backward(W.PrefillCase("bwd_bf16", 1, 2, 700, d, True), grad_dtype=torch.bfloat16)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 33, 129, 257, 1000])
+def test_backward_ragged_bf16_grads(N, causal):
+    # bf16 dK / dV at d = 128 leave through tensor stores of 32-row boxes, clipped at row N
+    parity.run_backward(W.PrefillCase(f"bwd_bf16_N{N}", 1, 3, N, 128, causal),
+                        grad_dtype=torch.bfloat16)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_backward_peaked_rows_f32_o(d):
     # 1% of key rows x8: near one-hot probability rows.  There D = dO . O cancels against the
@@ -78,6 +86,32 @@ def test_guard_bytes_untouched():
     ws = torch.empty(lib.fa_bwd_workspace_size(1, 2, 200, 64), dtype=torch.uint8, device="cuda")
     st = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), 0, do.data_ptr(),
                     lse.data_ptr(), *(b[pad:].data_ptr() for b in bufs), 1, 1, 2, 200, 64, 0, 0.0,
+                    ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert st == 0 and fa.device_status() == 0
+    for b in bufs:
+        assert torch.isnan(b[:pad]).all() and torch.isnan(b[pad + n:]).all()
+        assert torch.isfinite(b[pad:pad + n]).all()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_guard_bytes_untouched_bf16_grads(d):
+    # bf16 gradients written into the middle of NaN-filled buffers: nothing outside [B, H, N, d]
+    # changes, also where a key block's last 32-row box reaches past N
+    import exact_attention_158_b200 as fa
+    case = W.PrefillCase("bwd_guard_bf16", 1, 2, 200, d, False)
+    q, k, v = W.make_prefill(case, device="cuda")
+    do = W.make_dout(case, device="cuda")
+    o, lse = fa.fa_fwd(q, k, v)
+    n = q.numel()
+    pad = 4096
+    bufs = [torch.full((n + 2 * pad,), float("nan"), dtype=torch.bfloat16, device="cuda")
+            for _ in range(3)]
+    views = [b[pad:pad + n].view(q.shape) for b in bufs]
+    lib = fa.load_library()
+    ws = torch.empty(lib.fa_bwd_workspace_size(1, 2, 200, d), dtype=torch.uint8, device="cuda")
+    st = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), 0, do.data_ptr(),
+                    lse.data_ptr(), *(t.data_ptr() for t in views), 0, 1, 2, 200, d, 0, 0.0,
                     ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert st == 0 and fa.device_status() == 0
