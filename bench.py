@@ -31,6 +31,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -189,17 +190,20 @@ def barrier():
 _CPU_INPUTS = None
 
 
-def cpu_baseline(target_s: float = 12.0):
-    import numpy as np
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _oracle_rows_rate(qb, kb, vb, threads, target_s, rng, BH, N, d):
+    """Time the oracle over random (head, row) samples, half causal; returns (TFLOP/s, rows, s)."""
     from oracle import oracle as orc
-    global _CPU_INPUTS
-    BH, N, d = 8 * 16, 2048, 128
-    if _CPU_INPUTS is None:
-        q, k, v = W.make_prefill(W.prefill_cases()[0], device="cpu")
-        _CPU_INPUTS = tuple(W.bf16_bits(t).reshape(BH, N, d) for t in (q, k, v))
-    qb, kb, vb = _CPU_INPUTS
-    threads = orc.default_threads()
-    rng = np.random.default_rng(0)
     flops = 0.0
     rows = 0
     t0 = time.perf_counter()
@@ -213,9 +217,53 @@ def cpu_baseline(target_s: float = 12.0):
             flops += float(4.0 * d * vis.sum())
             rows += batch
     el = time.perf_counter() - t0
-    return {"value": flops / el / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{rows} query rows of {WORKLOAD} (half causal), fp64, {el:.1f} s; "
-                      "throughput scaled by the exact FLOPs of the sampled rows"}
+    return flops / el / 1e12, rows, el
+
+
+def cpu_baseline(target_s: float = 12.0, one_thread_s: float = 3.0):
+    """The fp64 oracle on this host: all its threads over a bounded row sample of the headline
+    workload (the reported value), plus a 1-thread figure on the same kind of sample."""
+    from oracle import oracle as orc
+    global _CPU_INPUTS
+    BH, N, d = 8 * 16, 2048, 128
+    if _CPU_INPUTS is None:
+        q, k, v = W.make_prefill(W.prefill_cases()[0], device="cpu")
+        _CPU_INPUTS = tuple(W.bf16_bits(t).reshape(BH, N, d) for t in (q, k, v))
+    qb, kb, vb = _CPU_INPUTS
+    threads = orc.default_threads()
+    rng = np.random.default_rng(0)
+    value, rows, el = _oracle_rows_rate(qb, kb, vb, threads, target_s, rng, BH, N, d)
+    out = {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+           "sample": f"{rows} query rows of {WORKLOAD} (half causal), fp64, {el:.1f} s; "
+                     "throughput scaled by the exact FLOPs of the sampled rows",
+           "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+    if one_thread_s > 0:
+        v1, rows1, el1 = _oracle_rows_rate(qb, kb, vb, 1, one_thread_s, rng, BH, N, d)
+        out["value_1thread"] = v1
+        out["sample_1thread"] = f"{rows1} query rows, 1 thread, {el1:.1f} s"
+    return out
+
+
+def cpu_sweep_point(case, target_s: float = 0.25):
+    """The oracle (all host threads) on sampled rows of two (b, h) slices of one sweep point, its
+    time extrapolated to the whole point by the exact FLOPs of the sampled rows."""
+    from oracle import oracle as orc
+    heads = [0, case.B * case.H - 1]
+    q, k, v = (W.bf16_bits(t) for t in W.make_prefill_heads(case, heads))
+    threads = orc.default_threads()
+    rng = np.random.default_rng(1)
+    flops, rows, t0 = 0.0, 0, time.perf_counter()
+    batch = max(32, threads * 4)
+    while time.perf_counter() - t0 < target_s:
+        pairs = np.stack([rng.integers(0, 2, batch), rng.integers(0, case.N, batch)], 1)
+        orc.attention_rows(q, k, v, case.causal, case.scale, pairs, threads)
+        vis = (pairs[:, 1] + 1) if case.causal else np.full(batch, case.N)
+        flops += float(4.0 * case.d * vis.sum())
+        rows += batch
+    el = time.perf_counter() - t0
+    tf = flops / el / 1e12
+    return {"tflops": tf, "ms_extrapolated": case.flops / (tf * 1e12) * 1e3, "rows": rows,
+            "cores": threads, "extrapolated": True}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -251,12 +299,27 @@ def bench_decode(fa, args, dev, flush, stream, pk):
     ms = statistics.median(ts)
     nbytes = W.decode_bytes(inp["lens"], case.H, case.d, inp["max_blocks"])
     gbs = nbytes / (ms * 1e-3) / 1e9
+    # the decode only reads: its denominator is the read-only bandwidth measured here with the
+    # same streaming loads over a 4 GiB buffer (best of five), besides the copy figure
+    tokens = sum(inp["lens"])
+    del inp, o, lse, ws
+    torch.cuda.empty_cache()
+    rbuf = torch.empty(4 << 30, dtype=torch.uint8, device=dev)
+    fa.probe_read_rate(rbuf)
+    read_gbs = max(rbuf.numel() / (fa.probe_read_rate(rbuf) * 1e-3) / 1e9 for _ in range(5))
+    del rbuf
+    torch.cuda.empty_cache()
     return {"metric": "paged decode GB/s", "workload": f"{case.S} seqs, q len 1, H32 d128, "
             "context U[512,8192], 16-token pages, permuted block table",
             "ms": round(ms, 4), "value": round(gbs, 1), "unit": "GB/s",
-            "algorithmic_bytes": nbytes, "tokens": sum(inp["lens"]),
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+            "algorithmic_bytes": nbytes, "tokens": tokens,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(read_gbs, 1),
+                         "unit": "GB/s", "frac": round(gbs / read_gbs, 4),
+                         "peak_source": "read-only bandwidth measured in this run "
+                                        "(fa_probe_read_rate, 4 GiB, best of 5)",
+                         "frac_of_copy_peak": round(gbs / pk["hbm_gbs"], 4),
+                         "copy_peak": pk["hbm_gbs"],
+                         "frac_of_nominal_7700": round(gbs / 7700.0, 4),
                          "traffic": committed_traffic("decode", DECODE_SOURCES)},
             "launches_per_step": 2}
 
@@ -413,6 +476,21 @@ def bench_backward(fa, args, dev, flush, stream, pk):
             "roofline": {"bound": "tensor", "achieved": round(tot_tf, 1), "peak": pk["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": round(tot_tf / pk["bf16_tflops"], 4)},
             "launches_per_step": 6}
+
+
+def measure_ex2(fa, dev):
+    """Exponentials per second on the special-function unit (best of three ~0.1 s probes), and
+    per SM per clock at the SM clock sampled meanwhile."""
+    fa.probe_ex2_rate(2000)
+    with ClockSampler(dev.index) as clk:
+        best = max(n / (ms * 1e-3) for n, ms in (fa.probe_ex2_rate(200_000) for _ in range(3)))
+    c = clk.summary()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = c["sm_mhz"] or c["sm_max_mhz"]
+    return {"exps_per_s": best, "sms": sms, "sm_mhz": mhz,
+            "per_sm_per_clk": round(best / (sms * mhz * 1e6), 3) if mhz else None,
+            "how": "fa_probe_ex2_rate: 4 CTAs x 256 threads per SM, 16 independent ex2 chains "
+                   "per thread, CUDA events; one exponential per 4 d FLOP of the forward"}
 
 
 def bench_ours(args, rank, world):
@@ -572,20 +650,43 @@ def bench_ours(args, rank, world):
     torch.cuda.empty_cache()
 
     # ---- sequence-length sweep (the pages' benchmark grid)
-    sweep = []
+    # Ceilings per point: the dense bf16 peak, HBM (algorithmic bytes x measured bandwidth) and the
+    # exponentials (one per 4 d FLOP, at the special-function unit's rate measured on this GPU by
+    # fa_probe_ex2_rate, scaled to the SM clock sampled during the sweep).
+    sweep, mufu = [], None
     if not args.no_sweep:
-        for d in (128, 64):
-            for case in W.sweep_cases(d):
-                ts = run_prefill_case(fa, case, args.sweep_steps, 3, flush, stream)
-                ms = statistics.median(ts)
-                tf = case.flops / (ms * 1e-3) / 1e12
-                intensity = case.flops / (4 * case.B * case.H * case.N * case.d * 2 + case.B * case.H * case.N * 4)
-                attainable = min(pk["bf16_tflops"], intensity * pk["hbm_gbs"] / 1e3)
-                sweep.append({"d": d, "N": case.N, "B": case.B, "H": case.H, "causal": case.causal,
-                              "ms": round(ms, 4), "tflops": round(tf, 1),
-                              "frac_peak": round(tf / pk["bf16_tflops"], 4),
-                              "frac_attainable": round(tf / attainable, 4)})
-                torch.cuda.empty_cache()
+        mufu = measure_ex2(fa, dev)
+        with ClockSampler(dev.index) as sclk:
+            for d in (128, 64):
+                for case in W.sweep_cases(d):
+                    ts = run_prefill_case(fa, case, args.sweep_steps, 3, flush, stream)
+                    sweep.append((case, statistics.median(ts)))
+                    torch.cuda.empty_cache()
+        sweep_mhz = sclk.summary()["sm_mhz"] or mufu["sm_mhz"]
+        mufu["sweep_sm_mhz"] = sweep_mhz
+        rows = []
+        for case, ms in sweep:
+            tf = case.flops / (ms * 1e-3) / 1e12
+            intensity = case.flops / (4 * case.B * case.H * case.N * case.d * 2 + case.B * case.H * case.N * 4)
+            hbm_ceiling = intensity * pk["hbm_gbs"] / 1e3
+            if mufu["per_sm_per_clk"] and sweep_mhz:
+                exps_s = mufu["per_sm_per_clk"] * mufu["sms"] * sweep_mhz * 1e6
+            else:
+                exps_s = mufu["exps_per_s"]
+            mufu_ceiling = exps_s * 4 * case.d / 1e12
+            attainable = min(pk["bf16_tflops"], hbm_ceiling, mufu_ceiling)
+            row = {"d": case.d, "N": case.N, "B": case.B, "H": case.H, "causal": case.causal,
+                   "ms": round(ms, 4), "tflops": round(tf, 1),
+                   "frac_peak": round(tf / pk["bf16_tflops"], 4),
+                   "mufu_ceiling_tflops": round(mufu_ceiling, 1),
+                   "frac_mufu": round(tf / mufu_ceiling, 4),
+                   "frac_attainable": round(tf / attainable, 4),
+                   "bound_by": ("tensor" if attainable == pk["bf16_tflops"] else
+                                "hbm" if attainable == hbm_ceiling else "mufu")}
+            if not args.no_cpu_baseline and rank == 0:
+                row["cpu_oracle"] = cpu_sweep_point(case)
+            rows.append(row)
+        sweep = rows
 
     # ---- paged decode (HBM bound)
     dec = None if args.no_decode else bench_decode(fa, args, dev, flush, stream, pk)
@@ -603,7 +704,7 @@ def bench_ours(args, rank, world):
     seqpar = (None if args.no_seqpar else
               bench_sequence_parallel(fa, args, dev, flush, stream, pk, rank, world))
 
-    result.update({"e2e": e2e, "sweep": sweep, "decode": dec, "paged_prefill": paged,
+    result.update({"e2e": e2e, "sweep": sweep, "mufu": mufu, "decode": dec, "paged_prefill": paged,
                    "backward": bwd, "tree": tree, "sequence_parallel": seqpar})
     return result
 

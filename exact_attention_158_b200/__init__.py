@@ -33,7 +33,8 @@ EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
                     "fa_bwd_workspace_size",
                     "fa_bwd", "fa_get_device_status",
                     "fa_status_string",
-                    "fa_last_error_string", "fa_version", "fa_selftest_wait_timeout")
+                    "fa_last_error_string", "fa_version", "fa_selftest_wait_timeout",
+                    "fa_probe_ex2_rate", "fa_probe_read_rate")
 
 _lib = None
 
@@ -376,12 +377,34 @@ def fa_decode_paged_noalloc(q, k_pool, v_pool, block_table, seq_lens, out, lse=N
         _require(t, n)
     _require(block_table, "block_table", torch.int32)
     _require(seq_lens, "seq_lens", torch.int32)
-    _require(out, "out", out.dtype)
+    if q.dim() != 3:
+        raise ValueError("q must be [S, H, d]")
     S, H, d = q.shape
-    st = f(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),
-           block_table.shape[1], seq_lens.data_ptr(), k_pool.shape[0], out.data_ptr(),
-           _out_code(out.dtype), lse.data_ptr() if lse is not None else None, S, H, d,
-           float(scale) if scale is not None else 0.0, _stream_handle(stream))
+    P = k_pool.shape[0]
+    if k_pool.shape != (P, H, 16, d) or v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool / v_pool must be [num_blocks, H, 16, d]")
+    if block_table.dim() != 2 or block_table.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_table must be [S, max_blocks] and seq_lens [S]")
+    code = _out_code(out.dtype) if isinstance(out, torch.Tensor) else None
+    if code is None:
+        raise ValueError("out must be a bf16 or fp32 CUDA tensor")
+    _require(out, "out", out.dtype)
+    if out.shape != (S, H, d):
+        raise ValueError("out must be [S, H, d]")
+    if lse is not None:
+        _require(lse, "lse", torch.float32)
+        if lse.shape != (S, H):
+            raise ValueError("lse must be [S, H]")
+    for t, n in ((k_pool, "k_pool"), (v_pool, "v_pool"), (block_table, "block_table"),
+                 (seq_lens, "seq_lens"), (out, "out")) + (((lse, "lse"),) if lse is not None else ()):
+        if t.device != q.device:
+            raise ValueError(f"{n} must be on q's device ({q.device})")
+    # the library resolves its scratch array, and launches, on the current device
+    with torch.cuda.device(q.device):
+        st = f(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(),
+               block_table.shape[1], seq_lens.data_ptr(), P, out.data_ptr(), code,
+               lse.data_ptr() if lse is not None else None, S, H, d,
+               float(scale) if scale is not None else 0.0, _stream_handle(stream))
     _check(st, "fa_decode_paged_noalloc")
     return out, lse
 
@@ -395,3 +418,41 @@ def selftest_wait_timeout(limit_us: int = 50_000, stream=None) -> int:
     f.restype = ctypes.c_int
     _check(f(limit_us, _stream_handle(stream)), "fa_selftest_wait_timeout")
     return device_status(stream)
+
+
+def probe_ex2_rate(iters: int = 200_000, stream=None) -> tuple[int, float]:
+    """Run the exponential-throughput probe once on the current device; returns (exponentials
+    launched, device milliseconds from CUDA events on the stream)."""
+    lib = load_library()
+    f = lib.fa_probe_ex2_rate
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_longlong), ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    s = stream if stream is not None else torch.cuda.current_stream()
+    sink = torch.zeros(1, dtype=torch.float32, device="cuda")
+    n = ctypes.c_longlong(0)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    _check(f(sink.data_ptr(), int(iters), ctypes.byref(n), int(s.cuda_stream)), "fa_probe_ex2_rate")
+    b.record(s)
+    b.synchronize()
+    return int(n.value), a.elapsed_time(b)
+
+
+def probe_read_rate(buf: torch.Tensor, stream=None) -> float:
+    """Read every byte of the contiguous CUDA tensor `buf` once with the decode's streaming loads;
+    returns the device milliseconds (CUDA events on the stream)."""
+    lib = load_library()
+    f = lib.fa_probe_read_rate
+    f.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise ValueError("buf must be a contiguous CUDA tensor")
+    s = stream if stream is not None else torch.cuda.current_stream()
+    sink = torch.zeros(1, dtype=torch.float32, device=buf.device)
+    nbytes = buf.numel() * buf.element_size()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    _check(f(buf.data_ptr(), nbytes, sink.data_ptr(), int(s.cuda_stream)), "fa_probe_read_rate")
+    b.record(s)
+    b.synchronize()
+    return a.elapsed_time(b)

@@ -30,6 +30,42 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   fence_mbar_init();
   mbar_wait(&bar, 0, &abort_flag, limit_ns);  // records FA_ERR_TIMEOUT when it gives up
 }
+
+// MUFU throughput probe: every thread runs kEx2Chains independent chains x <- 2^x - 1.5 (which
+// stays in [-1.5, 0.5]), so the exponentials, not their latency, bound the kernel.  The sink is
+// written only if the sum takes a value it never takes, which keeps the work alive.
+constexpr int kEx2Chains = 16;
+__global__ void __launch_bounds__(256) ex2_rate_kernel(float *sink, int iters) {
+  float x[kEx2Chains];
+#pragma unroll
+  for (int i = 0; i < kEx2Chains; ++i) x[i] = -1.f + 1e-2f * i + 1e-5f * threadIdx.x;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int i = 0; i < kEx2Chains; ++i) x[i] = ex2(x[i]) - 1.5f;
+  }
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < kEx2Chains; ++i) acc += x[i];
+  if (acc == 1.0e30f) *sink = acc;
+}
+
+// HBM read probe: a grid-stride sweep over the buffer with the decode kernel's 16-byte streaming
+// loads, four in flight per thread; the words are xor-folded so the loads stay live.
+__global__ void __launch_bounds__(512) read_rate_kernel(const uint4 *buf, size_t n16, float *sink) {
+  uint32_t acc = 0;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    uint4 a = ld_stream_v4(buf + i), b = ld_stream_v4(buf + i + stride);
+    uint4 c = ld_stream_v4(buf + i + 2 * stride), d = ld_stream_v4(buf + i + 3 * stride);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w ^ b.x ^ b.y ^ b.z ^ b.w ^ c.x ^ c.y ^ c.z ^ c.w ^ d.x ^ d.y ^ d.z ^ d.w;
+  }
+  for (; i < n16; i += stride) {
+    uint4 a = ld_stream_v4(buf + i);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w;
+  }
+  if (acc == 0x7fc01234u) *sink = __uint_as_float(acc);
+}
 }  // namespace fa
 
 namespace {
@@ -754,6 +790,32 @@ fa_status fa_selftest_wait_timeout(unsigned limit_us, fa_stream_t stream) {
   if (st != FA_OK) return st;
   fa::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(limit_us) * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : launch_failed(e);
+}
+
+fa_status fa_probe_ex2_rate(float *sink, int iters, long long *exps_out, fa_stream_t stream) {
+  if (!sink || !exps_out || iters < 1 || iters > (1 << 24)) return FA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  const int blocks = 4 * dev->num_sms;  // 32 warps per SM: 8 per sub-partition
+  fa::ex2_rate_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(sink, iters);
+  *exps_out = static_cast<long long>(blocks) * 256 * iters * fa::kEx2Chains;
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : launch_failed(e);
+}
+
+fa_status fa_probe_read_rate(const void *buf, size_t bytes, float *sink, fa_stream_t stream) {
+  if (!buf || !sink || bytes < 16 || bytes % 16) return FA_ERR_INVALID_ARG;
+  if (!aligned16(buf)) return FA_ERR_ALIGNMENT;
+  DeviceInfo *dev = nullptr;
+  int dev_id = 0;
+  fa_status st = current_device(&dev, &dev_id);
+  if (st != FA_OK) return st;
+  fa::read_rate_kernel<<<4 * dev->num_sms, 512, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4 *>(buf), bytes / 16, sink);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : launch_failed(e);
 }

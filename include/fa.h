@@ -131,8 +131,8 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *
  *   q, k, v, dout     bf16 [B, H, N, d] contiguous, 16-byte aligned; dout is the incoming gradient.
  *   o, o_dtype        fa_fwd's output for the same q, k, v, causal and scale, [B, H, N, d] in bf16
- *                     or fp32.  D is formed from it, so bf16 O carries its own rounding (2^-9
- *                     relative) into dS; fp32 O avoids that where rows are nearly one-hot.
+ *                     or fp32.  D is formed from it, so bf16 O carries its own rounding (up to
+ *                     2^-8 relative) into dS; fp32 O avoids that where rows are nearly one-hot.
  *   lse               fp32 [B, H, N], fa_fwd's log-sum-exp for the same call.
  *   dq, dk, dv        [B, H, N, d], bf16 or fp32 per g_dtype, 16-byte aligned; must not overlap the
  *                     inputs, one another or the workspace.
@@ -255,8 +255,11 @@ fa_status fa_tree_attention(const void *q, const void *k_pool, const void *v_poo
  *
  * The scratch is a static device array of FA_NOALLOC_SCRATCH_BYTES inside this library: every
  * GPU that loads the library holds it until the process exits.  The first call on each device
- * looks up the array's device address (cudaGetSymbolAddress, no allocation); make that first call
- * before any stream capture.  Arguments are as for fa_decode_paged; sizes whose
+ * looks up the array's device address (cudaGetSymbolAddress, no allocation) and keeps it for the
+ * life of the process; make that first call before any stream capture.  A device reset
+ * (cudaDeviceReset, or the primary context destroyed and created again) makes the kept address
+ * stale: do not call this entry point again in a process after resetting a device it has run on.
+ * Arguments are as for fa_decode_paged; sizes whose
  * fa_decode_workspace_size(S, H, d, max_blocks_per_seq) exceeds FA_NOALLOC_SCRATCH_BYTES return
  * FA_ERR_WORKSPACE (fa_last_error_string() says how many bytes were needed) and launch nothing.
  * No slot of the array needs to start at zero: every slot a call reads was written earlier in
@@ -286,6 +289,29 @@ fa_status fa_get_device_status(fa_stream_t stream);
  * a stalled kernel is reported through fa_get_device_status instead of hanging the GPU.
  */
 fa_status fa_selftest_wait_timeout(unsigned limit_us, fa_stream_t stream);
+
+/*
+ * fa_probe_ex2_rate -- diagnostic: launches a kernel (4 CTAs of 256 threads per SM) whose threads
+ * each evaluate `iters` x 16 base-2 exponentials on the special-function unit, the instruction the
+ * online softmax uses for p = 2^(s * scale * log2 e - m) ("Flash Attention" (myungum), section 2,
+ * the exponentials of each score block).  Writes the number of exponentials launched to *exps_out
+ * (host memory); the caller times the launch on `stream` and divides.  The result is the ceiling
+ * that the exponentials put on the forward: one per 4 d FLOP of Q K^T and P V.  `sink` is one
+ * float of device memory the kernel may write (it never does for these inputs).  iters in
+ * 1 .. 2^24, else FA_ERR_INVALID_ARG.
+ */
+fa_status fa_probe_ex2_rate(float *sink, int iters, long long *exps_out, fa_stream_t stream);
+
+/*
+ * fa_probe_read_rate -- diagnostic: reads `bytes` (a multiple of 16, >= 16) of device memory at
+ * `buf` (16-byte aligned) once, with the 16-byte streaming loads the paged decode uses to walk the
+ * KV cache ("LLM study notes", paged attention: decode reads every cached key and value), from
+ * 4 CTAs of 512 threads per SM.  The caller times the launch on `stream`: bytes / time is the
+ * read-only HBM bandwidth that bounds the decode, which only reads.  `sink` is one float of device
+ * memory the kernel may write.  Bad sizes or pointers return FA_ERR_INVALID_ARG /
+ * FA_ERR_ALIGNMENT before anything launches.
+ */
+fa_status fa_probe_read_rate(const void *buf, size_t bytes, float *sink, fa_stream_t stream);
 
 /* Static text for a status code. */
 const char *fa_status_string(fa_status status);

@@ -126,3 +126,15 @@ def test_tree_verify_flops_counts_visible_pairs():
                 anc, u = anc + 1, p[u]
             pairs += (L - 4) + anc
     assert W.tree_verify_flops(lens, masks, 3, 8) == 4 * 8 * 3 * pairs
+
+
+def test_head_subset_generator_matches_full_tensors():
+    # the bench's per-point oracle samples draw only a few (b, h) slices; they must be the very
+    # slices the full generator produces, peaked and rising variants included
+    for case in (W.PrefillCase("h", 2, 3, 300, 64, False, peaked=True),
+                 W.PrefillCase("h", 1, 2, 1000, 128, True, rising=True)):
+        full = W.make_prefill(case)
+        heads = [0, case.B * case.H - 1]
+        part = W.make_prefill_heads(case, heads)
+        for a, b in zip(full, part):
+            assert torch.equal(a.reshape(-1, case.N, case.d)[heads], b)

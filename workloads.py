@@ -81,8 +81,12 @@ def _top53(w: torch.Tensor) -> torch.Tensor:
     return _lsr(w, 11).to(torch.float64)
 
 
-def normal_bf16(seed: int, tensor_id: int, numel: int, device="cpu", chunk: int = 1 << 26) -> torch.Tensor:
-    """``numel`` N(0,1) draws rounded to bf16, element i of the stream at flat index i."""
+def normal_bf16(seed: int, tensor_id: int, numel: int, device="cpu", chunk: int = 1 << 26,
+                first: int = 0) -> torch.Tensor:
+    """``numel`` N(0,1) draws rounded to bf16: elements first .. first+numel-1 of the stream
+    (``first`` even, so that Box-Muller pairs line up with the full tensor's)."""
+    if first % 2:
+        raise ValueError("first must be even")
     out = torch.empty(numel, dtype=torch.bfloat16, device=device)
     two53 = float(1 << 53)
     start = 0
@@ -90,7 +94,7 @@ def normal_bf16(seed: int, tensor_id: int, numel: int, device="cpu", chunk: int 
         # pairs must start on an even index
         n = min(chunk, numel - start)
         npair = (n + 1) // 2
-        w = raw_words(seed, tensor_id, start, 2 * npair, device)
+        w = raw_words(seed, tensor_id, first + start, 2 * npair, device)
         w = w.view(npair, 2)
         u1 = (_top53(w[:, 0]) + 1.0) / two53
         u2 = _top53(w[:, 1]) / two53
@@ -130,8 +134,10 @@ class PrefillCase:
     N: int
     d: int
     causal: bool
-    peaked: bool = False          # 1 % of key rows of every (b, h) scaled by 8
+    peaked: bool = False          # 1 % of key rows of every (b, h) scaled by peak_factor
+    peak_factor: int = 8          # a power of two, so the scaled bf16 rows are exact
     seed: int = BASE_SEED
+    rising: bool = False          # key blocks scaled by rising_factor (x1, then x8, then x64)
 
     @property
     def scale(self) -> float:
@@ -159,6 +165,16 @@ def peaked_rows(seed: int, bh: int, N: int) -> list[int]:
     return sorted(idx[:r])
 
 
+def rising_factor(pos: int, n: int) -> int:
+    """Scale of the key at position ``pos`` of a length-``n`` sequence in the "rising" inputs: its
+    128-key block b of nb = ceil(n/128) gets 1 in the first third (3b < nb), 8 in the second
+    (3b < 2nb) and 64 in the last.  Powers of two, so the scaled bf16 keys are exact; the row
+    maxima of the scores then jump by far more than 2^8 (in log2 units) after the first block."""
+    nb = -(-n // 128)
+    b = pos // 128
+    return 1 if 3 * b < nb else (8 if 3 * b < 2 * nb else 64)
+
+
 def make_prefill(case: PrefillCase, device="cpu"):
     """Q, K, V as bf16 tensors of shape [B, H, N, d] (contiguous), on ``device``."""
     shape = (case.B, case.H, case.N, case.d)
@@ -170,7 +186,32 @@ def make_prefill(case: PrefillCase, device="cpu"):
         kf = k.view(case.B * case.H, case.N, case.d)
         for bh in range(case.B * case.H):
             rows = torch.tensor(peaked_rows(case.seed, bh, case.N), device=device)
-            kf[bh, rows] = kf[bh, rows] * 8  # power of two: exact in bf16
+            kf[bh, rows] = kf[bh, rows] * case.peak_factor  # power of two: exact in bf16
+    if case.rising:
+        f = torch.tensor([rising_factor(p, case.N) for p in range(case.N)], dtype=torch.bfloat16,
+                         device=device)
+        k.mul_(f.view(1, 1, case.N, 1))
+    return q, k, v
+
+
+def make_prefill_heads(case: PrefillCase, heads, device="cpu"):
+    """Q, K, V of the listed (b, h) slices only (flat index bh = b * H + h), as bf16 tensors
+    [len(heads), N, d]: the same values make_prefill gives those slices, without drawing the rest."""
+    N, d = case.N, case.d
+    out = []
+    for tid in (TID_Q, TID_K, TID_V):
+        t = torch.stack([normal_bf16(case.seed, tid, N * d, device, first=bh * N * d).view(N, d)
+                         for bh in heads])
+        out.append(t)
+    q, k, v = out
+    for i, bh in enumerate(heads):
+        if case.peaked:
+            rows = torch.tensor(peaked_rows(case.seed, bh, N), device=device)
+            k[i, rows] = k[i, rows] * case.peak_factor
+    if case.rising:
+        f = torch.tensor([rising_factor(p, N) for p in range(N)], dtype=torch.bfloat16,
+                         device=device)
+        k.mul_(f.view(1, N, 1))
     return q, k, v
 
 
@@ -209,6 +250,7 @@ class DecodeCase:
     len_hi: int = 8192
     seed: int = BASE_SEED
     lens: list = field(default=None)  # optional explicit context lengths
+    rising: bool = False        # keys scaled by rising_factor of their position in the sequence
 
     @property
     def scale(self) -> float:
@@ -249,6 +291,14 @@ def make_decode(case: DecodeCase, device="cpu"):
     q = normal_bf16(case.seed, TID_Q, case.S * case.H * case.d, device).view(case.S, case.H, case.d)
     k_pool = normal_bf16(case.seed, TID_K, P * page_elems, device).view(P, case.H, PAGE_SIZE, case.d)
     v_pool = normal_bf16(case.seed, TID_V, P * page_elems, device).view(P, case.H, PAGE_SIZE, case.d)
+    if case.rising:
+        # 128-key blocks start on page boundaries, so one factor covers a whole page
+        for s in range(case.S):
+            for pg in range(nblk[s]):
+                f = rising_factor(pg * PAGE_SIZE, lens[s])
+                if f != 1:
+                    blk = int(table[s, pg])
+                    k_pool[blk] = k_pool[blk] * f
     for s in range(case.S):
         tail = lens[s] % PAGE_SIZE
         if tail:
