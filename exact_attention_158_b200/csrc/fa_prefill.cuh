@@ -53,6 +53,12 @@ constexpr float kLn2 = 0.6931471805599453f;
 #endif
 // every FA_POLY_EVERY-th pair of P's exponentials on the FMA pipe, the rest on MUFU (0: all MUFU)
 constexpr int kPolyEvery = FA_POLY_EVERY;
+#ifndef FA_TWO_ISSUERS
+#define FA_TWO_ISSUERS 1
+#endif
+#ifndef FA_EXP_TURNS
+#define FA_EXP_TURNS 1
+#endif
 
 template <int HD>
 struct PrefillCfg {
@@ -66,6 +72,17 @@ struct PrefillCfg {
   // MMA issue order: at d = 64 an event-driven loop (issue whatever S or P V is ready) measured
   // faster; at d = 128 the fixed order S_0,j+1  S_1,j+1  PV_0,j  PV_1,j did.
   static constexpr bool kEventMma = HD == 64;
+  // Two MMA-issuing threads (Q K^T from warp 9, P V from warp 10) instead of one: the tensor core
+  // accepts only about one MMA ahead of its issuer, so whatever an issuer does between groups
+  // (barrier waits, commits) idles it unless the other issuer has work to hand over meanwhile.
+  static constexpr bool kTwoIssuers = FA_TWO_ISSUERS != 0;
+  // Exponential turns: softmax warp w (tile 0) and warp w + 4 (tile 1) run on the same SM
+  // sub-partition and share its special-function unit, which evaluates a row block's 128
+  // exponentials per thread about as fast as the tensor core does the block's MMAs.  Left to
+  // themselves the two warps fall into step and slow each other's exponentials; taking turns (one
+  // warp's exponentials while the other loads scores, finds its maximum and stores P) keeps the
+  // unit busy without contention.
+  static constexpr bool kExpTurns = FA_EXP_TURNS != 0;
   static constexpr int kPBytes = kPInTmem ? 0 : 128 * kBN * 2;  // one 128 x 128 bf16 P tile
   // bf16 O staging for the tensor-store epilogue: the P tile where there is one, else a buffer of
   // its own per query tile (d = 64: 128 rows x 128 bytes)
@@ -76,7 +93,7 @@ struct PrefillCfg {
   static constexpr int kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + HD;
   static constexpr uint32_t kColP0 = 256 + 2 * HD, kColP1 = kColP0 + kBN / 2;  // TMEM P (d = 64)
-  static constexpr int kNumBars = 2 + 2 * kStages + 4 * 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kStages + 4 * 2 + 2 + 8;
   static constexpr int kSchedBytes = 2 * 128 * 4;  // paged mode: sequence lengths and their order
   static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + 2 * kTileBytes +
                                        kStages * kTileBytes + 2 * kPBytes + 2 * kOStageBytes +
@@ -197,16 +214,20 @@ __device__ __forceinline__ int tile_blocks(const PrefillParams &p, const KvSpan 
   return last_key / kBN + 1;
 }
 
+// The tensor core takes a new MMA only about as fast as it completes one, so the issuing thread
+// runs in step with it: every instruction between two MMAs is tensor-core idle time.  The
+// descriptors of a group are therefore formed once, and each MMA adds a constant to them: for an
+// address below 2^18 (all of shared memory), desc(addr + off) = desc(addr) + off / 16 exactly.
+
 // S (TMEM) = Q (smem, K-major) K^T (smem, K-major), K = HD in steps of 16.
 template <int HD>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
   using C = PrefillCfg<HD>;
+  const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024), kd = smem_desc_sw128(k_smem, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
-    const uint32_t off = (kk / 4) * C::kChunkBytes + (kk % 4) * 32;
-    const uint64_t a = smem_desc_sw128(q_smem + off, 16, 1024);
-    const uint64_t b = smem_desc_sw128(k_smem + off, 16, 1024);
-    umma_ss(d_tmem, a, b, C::kIdescQK, kk > 0 ? 1u : 0u);
+    const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kChunkBytes + (kk % 4) * 32) >> 4);
+    umma_ss(d_tmem, qd + off, kd + off, C::kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -218,15 +239,16 @@ template <int HD>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_addr, uint32_t v_smem,
                                          bool accumulate) {
   using C = PrefillCfg<HD>;
+  const uint64_t vd = smem_desc_sw128(v_smem, C::kChunkBytes, 1024);
+  const uint64_t pd = C::kPInTmem ? 0 : smem_desc_sw128(p_addr, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk) {
-    const uint64_t b = smem_desc_sw128(v_smem + kk * 16 * 128, C::kChunkBytes, 1024);
+    const uint64_t b = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
     if constexpr (C::kPInTmem) {
       umma_ts(o_tmem, p_addr + kk * 8, b, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
     } else {
-      const uint32_t off = (kk / 4) * C::kChunkBytes + (kk % 4) * 32;
-      const uint64_t a = smem_desc_sw128(p_addr + off, 16, 1024);
-      umma_ss(o_tmem, a, b, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+      const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kChunkBytes + (kk % 4) * 32) >> 4);
+      umma_ss(o_tmem, pd + off, b, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
     }
   }
 }
@@ -338,8 +360,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t *s_free = s_full + 2;             // [2] S_i copied out by the softmax (4 warp arrivals)
   uint64_t *p_full = s_free + 2;             // [2] P_i written to smem (4 warp arrivals)
   uint64_t *pv_done = p_full + 2;            // [2] O_i += P_i V finished (MMA commit)
-  uint64_t *drain = pv_done + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *drain = pv_done + 2;             // [2] every MMA of issuer 0 / 1 has completed
+  uint64_t *turn = drain + 2;                // [8] exponential turns: [k] warp k, [4 + k] warp 4 + k
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(turn + 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *s_lens = const_cast<int *>(reinterpret_cast<volatile int *>(abort_flag + 1));  // [128]
   int *s_order = s_lens + kMaxSortedSeqs;                                              // [128]
@@ -363,7 +386,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(&p_full[i], kBM / 32);
       mbar_init(&pv_done[i], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
+    for (int k = 0; k < 8; ++k) mbar_init(&turn[k], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -479,6 +504,80 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (q_issued) mbar_wait(q_full, q_ph ^ 1, &never);
       }
     }
+  } else if (C::kTwoIssuers && (warp == 9 || warp == 10)) {
+    // ------------------------------------------------------------------ MMA issuers (two)
+    // Warp 9 issues S_i,j = Q_i K_j^T, warp 10 issues O_i += P_i,j V_j, each in block order and
+    // each committing its own barriers; K_j's stage is released by the first, V_j's by the second.
+    // Per unit the loads arrive in the order K_0, then K_{j+1}, V_j for j = 0, 1, ...: load index
+    // of K_j is 2j-1 (K_0: 0), of V_j 2j+2 (2j+1 for the last block).  A stage is reloaded only
+    // after the issuer that waits on its previous load has released it, so a parity wait can never
+    // see a phase two steps ahead.
+    if (lane == 0) {
+      const bool scores = warp == 9;
+      uint32_t kv_base = 0, q_ph = 0;
+      uint32_t s_cnt[2] = {0, 0};  // S_i computed so far (s_free phases follow it)
+      uint32_t p_cnt[2] = {0, 0};  // P_i consumed so far (p_full phases follow it)
+      const uint32_t sQ0 = smem_u32(sQ), sQ1 = smem_u32(sQ + C::kTileBytes);
+      const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_for_round<kGeneral>(p, r, seq_order);
+        if (u < 0) break;
+        const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
+        const KvSpan kv = kv_span<kMode>(p, w.bh);
+        const int n[2] = {tile_blocks(p, kv, w.pair, 0), tile_blocks(p, kv, w.pair, 1)};
+        const int nmax = n[0] > n[1] ? n[0] : n[1];
+        if (scores) {
+          if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
+          q_ph ^= 1;
+          for (int j = 0; ok && j < nmax; ++j) {
+            const uint32_t ld = kv_base + (j == 0 ? 0u : static_cast<uint32_t>(2 * j - 1));
+            const uint32_t st = ld % C::kStages;
+            if (!mbar_wait(&kv_full[st], (ld / C::kStages) & 1, abort_flag)) { ok = false; break; }
+            for (int i = 0; i < 2; ++i) {
+              if (j >= n[i]) continue;
+              if (s_cnt[i] > 0 && !mbar_wait(&s_free[i], (s_cnt[i] - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_qk<HD>(tmem + (i ? C::kColS1 : C::kColS0), i ? sQ1 : sQ0,
+                           sKV0 + st * C::kTileBytes);
+              umma_commit(&s_full[i]);
+              ++s_cnt[i];
+            }
+            if (!ok) break;
+            umma_commit(&kv_empty[st]);  // K_j is free once both S_i,j have been computed
+          }
+          if (!ok) break;
+          umma_commit(q_empty);  // every Q K^T of the unit is issued
+        } else {
+          for (int j = 0; ok && j < nmax; ++j) {
+            const uint32_t ld = kv_base + static_cast<uint32_t>(j + 1 < nmax ? 2 * j + 2 : 2 * j + 1);
+            const uint32_t st = ld % C::kStages;
+            if (!mbar_wait(&kv_full[st], (ld / C::kStages) & 1, abort_flag)) { ok = false; break; }
+            for (int i = 0; i < 2; ++i) {
+              if (j >= n[i]) continue;
+              if (!mbar_wait(&p_full[i], p_cnt[i] & 1, abort_flag)) { ok = false; break; }
+              ++p_cnt[i];
+              tc_fence_after();
+              const uint32_t p_addr = C::kPInTmem ? tmem + (i ? C::kColP1 : C::kColP0)
+                                                  : sP0 + i * C::kPBytes;
+              issue_pv<HD>(tmem + (i ? C::kColO1 : C::kColO0), p_addr, sKV0 + st * C::kTileBytes,
+                           j > 0);
+              umma_commit(&pv_done[i]);
+            }
+            if (!ok) break;
+            umma_commit(&kv_empty[st]);  // V_j is free once both P_i,j V_j have completed
+          }
+        }
+        kv_base += 2 * nmax;
+      }
+      // every MMA issued by this thread completes before TMEM is released
+      umma_commit(&drain[scores ? 0 : 1]);
+      volatile int never = 0;
+      mbar_wait(&drain[scores ? 0 : 1], 0, &never);
+    }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if constexpr (C::kEventMma) {
@@ -573,9 +672,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           kv_base += 2 * nmax;
         }
         // every MMA issued by this thread completes before TMEM is released
-        umma_commit(drain);
+        umma_commit(&drain[0]);
         volatile int never = 0;
-        mbar_wait(drain, 0, &never);
+        mbar_wait(&drain[0], 0, &never);
       }
     } else {
       if (lane == 0) {
@@ -646,9 +745,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
         }
         // every MMA issued by this thread completes before TMEM is released
-        umma_commit(drain);
+        umma_commit(&drain[0]);
         volatile int never = 0;
-        mbar_wait(drain, 0, &never);
+        mbar_wait(&drain[0], 0, &never);
       }
     }
   } else if (warp < 8) {
@@ -664,6 +763,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const float sl2 = p.scale_log2;
     uint32_t s_ph = 0, pv_ph = 0;
     bool ok = true;
+    // exponential turns with the warp of the other tile on this sub-partition (tile 0 first): wait
+    // on my barrier, run the exponentials, arrive on the other's.  Both warps take one turn per
+    // key block of the larger of the two tiles' block counts, so the turns always pair up.
+    uint64_t *turn_mine = turn + (wg ? 4 : 0) + warp % 4;
+    uint64_t *turn_other = turn + (wg ? 0 : 4) + warp % 4;
+    uint32_t turn_ph = 0;
+    auto take_turn = [&]() -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(turn_mine, turn_ph, abort_flag))) return false;
+      turn_ph ^= 1;
+      return true;
+    };
+    auto pass_turn = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(turn_other);
+    };
+    if (C::kExpTurns && wg == 1) pass_turn();
     for (int r = 0; ok; ++r) {
       const int u = unit_for_round<kGeneral>(p, r, seq_order);
       if (u < 0) break;
@@ -671,7 +786,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int pr = w.pair;
       const KvSpan kv = kv_span<kMode>(p, w.bh);
       const int n = tile_blocks(p, kv, pr, wg);
-      if (n == 0) continue;
+      const int n_other = tile_blocks(p, kv, pr, wg ^ 1);
+      if (n == 0) {
+        // a tile past the last query row: only its turns
+        if constexpr (C::kExpTurns) {
+          for (int j = 0; ok && j < n_other; ++j) {
+            if (!take_turn()) ok = false;
+            else pass_turn();
+          }
+        }
+        if (!ok) break;
+        continue;
+      }
       const int qrow = pr * 2 * kBM + wg * kBM + row;
       const bool tree = kPaged && p.tree_mask != nullptr;
       const uint64_t tmask =
@@ -735,8 +861,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
         uint32_t pk[kBN / 2];
+        if (C::kExpTurns && !take_turn()) { ok = false; break; }
         const float p_top = ex2(fmaf(s_top, sl2, mneg));
         const float le = FA_EXP_SCHEDULE ? exp_row_pipelined(s, sl2, mneg, pk) : exp_row(s, sl2, mneg, pk);
+        if (C::kExpTurns) pass_turn();
         // O is normalised by the sum of the bf16-rounded p that P V uses, so that it is a
         // convex combination of V rows even when one key dominates the row; the rounding error
         // that matters is the largest element's, so the fp32 sum is corrected by exactly that
@@ -785,6 +913,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[wg]);  // one arrival per warp
+      }
+      if (C::kExpTurns) {
+        // the other tile's extra block (causal pairs: tile 1 has one more)
+        for (int j = n; ok && j < n_other; ++j) {
+          if (!take_turn()) ok = false;
+          else pass_turn();
+        }
       }
       if (!ok) break;
       // epilogue: O_i / l and LSE once the last P V of this tile has completed
