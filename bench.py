@@ -89,7 +89,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples, self.reasons = [], set()
         self.max_mhz = None
         self._stop = threading.Event()

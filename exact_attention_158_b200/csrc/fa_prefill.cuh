@@ -48,14 +48,15 @@ constexpr int kBN = 128;  // keys per key/value block
 constexpr int kPrefillThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale: tolerate a stale max up to 2^8 below
 constexpr float kLn2 = 0.6931471805599453f;
+// every kPolyEvery-th pair of P's exponentials is evaluated on the FMA pipe, the rest on MUFU
+// (0: all MUFU).  At d = 128 every share tried (1/8 .. 1/2) was slower; at d = 64 a quarter was
+// about 7% faster but pushed peaked rows past the parity bound (max|dO| 1.25e-2 at N = 16k), so
+// both head dims use MUFU only.
 #ifndef FA_POLY_EVERY
 #define FA_POLY_EVERY 0
 #endif
-// every FA_POLY_EVERY-th pair of P's exponentials on the FMA pipe, the rest on MUFU (0: all MUFU)
+template <int HD>
 constexpr int kPolyEvery = FA_POLY_EVERY;
-#ifndef FA_TWO_ISSUERS
-#define FA_TWO_ISSUERS 1
-#endif
 #ifndef FA_EXP_TURNS
 #define FA_EXP_TURNS 1
 #endif
@@ -69,13 +70,6 @@ struct PrefillCfg {
   // P lives in TMEM when there is room for it beside S and O (d = 64: S 2x128 + O 2x64 + P 2x64
   // columns = 512), otherwise in shared memory (d = 128: S and O fill all 512 columns).
   static constexpr bool kPInTmem = HD == 64;
-  // MMA issue order: at d = 64 an event-driven loop (issue whatever S or P V is ready) measured
-  // faster; at d = 128 the fixed order S_0,j+1  S_1,j+1  PV_0,j  PV_1,j did.
-  static constexpr bool kEventMma = HD == 64;
-  // Two MMA-issuing threads (Q K^T from warp 9, P V from warp 10) instead of one: the tensor core
-  // accepts only about one MMA ahead of its issuer, so whatever an issuer does between groups
-  // (barrier waits, commits) idles it unless the other issuer has work to hand over meanwhile.
-  static constexpr bool kTwoIssuers = FA_TWO_ISSUERS != 0;
   // Exponential turns: softmax warp w (tile 0) and warp w + 4 (tile 1) run on the same SM
   // sub-partition and share its special-function unit, which evaluates a row block's 128
   // exponentials per thread about as fast as the tensor core does the block's MMAs.  Left to
@@ -93,7 +87,7 @@ struct PrefillCfg {
   static constexpr int kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + HD;
   static constexpr uint32_t kColP0 = 256 + 2 * HD, kColP1 = kColP0 + kBN / 2;  // TMEM P (d = 64)
-  static constexpr int kNumBars = 2 + 2 * kStages + 4 * 2 + 2 + 8;
+  static constexpr int kNumBars = 2 + 3 * kStages + 4 * 2 + 2 + 8;
   static constexpr int kSchedBytes = 2 * 128 * 4;  // paged mode: sequence lengths and their order
   static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + 2 * kTileBytes +
                                        kStages * kTileBytes + 2 * kPBytes + 2 * kOStageBytes +
@@ -256,6 +250,7 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_addr, uint3
 // One row of a score block -> P: p = 2^(s * scale*log2e - m_ref) for the 128 scores of this
 // thread's row (MUFU ex2, or the FMA-pipe polynomial for every kPolyEvery-th pair), packed to
 // bf16 pairs in pk.  Returns the sum of the fp32 p.
+template <int kPoly>
 __device__ __forceinline__ float exp_row(float (&s)[kBN], float sl2, float mneg,
                                          uint32_t (&pk)[kBN / 2]) {
   const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(mneg, mneg);
@@ -264,7 +259,7 @@ __device__ __forceinline__ float exp_row(float (&s)[kBN], float sl2, float mneg,
   for (int c = 0; c < kBN / 2; ++c) {
     const uint64_t x2 = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), c2, m2);
     uint64_t p2;
-    if (kPolyEvery > 0 && c % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+    if (kPoly > 0 && c % (kPoly > 0 ? kPoly : 1) == kPoly - 1) {
       p2 = exp2_poly_x2(x2);
     } else {
       float x0, x1;
@@ -354,8 +349,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(sO + 2 * C::kOStageBytes);
   uint64_t *q_full = bars;
   uint64_t *q_empty = bars + 1;
+  // kv_full[st]: a K tile has landed in stage st; kv_full[kStages + st]: a V tile has.  Each
+  // has one waiter (the Q K^T issuer for K, the P V issuer for V) that sees all of its phases
+  // in order, so a parity wait is exact: the next load of the same kind into the stage can only
+  // start after that waiter has consumed and released the current one.
   uint64_t *kv_full = bars + 2;
-  uint64_t *kv_empty = kv_full + C::kStages;
+  uint64_t *kv_empty = kv_full + 2 * C::kStages;
   uint64_t *s_full = kv_empty + C::kStages;  // [2] S_i computed (MMA commit)
   uint64_t *s_free = s_full + 2;             // [2] S_i copied out by the softmax (4 warp arrivals)
   uint64_t *p_full = s_free + 2;             // [2] P_i written to smem (4 warp arrivals)
@@ -378,6 +377,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(q_empty, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_full[C::kStages + s], 1);
       mbar_init(&kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -428,15 +428,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (lane == 0) {
       uint32_t kv_it = 0, q_ph = 0;
       bool q_issued = false;
-      uint32_t last_ph[C::kStages];
-      bool issued[C::kStages];
-      for (int s = 0; s < C::kStages; ++s) issued[s] = false;
+      uint32_t loads[2 * C::kStages];  // loads issued on each landing barrier (its phase count)
+      for (int b = 0; b < 2 * C::kStages; ++b) loads[b] = 0;
       bool ok = true;
       int kv_len = 0;  // key count of the current unit (paged mode)
-      auto load_kv = [&](const CUtensorMap *map, int row, int bh) -> bool {
+      auto load_kv = [&](const CUtensorMap *map, int row, int bh, bool is_v) -> bool {
         const uint32_t st = kv_it % C::kStages, ph = (kv_it / C::kStages) & 1;
         if (!mbar_wait(&kv_empty[st], ph ^ 1, abort_flag)) return false;
-        mbar_arrive_expect_tx(&kv_full[st], C::kTileBytes);
+        uint64_t *full = &kv_full[(is_v ? C::kStages : 0) + st];
+        mbar_arrive_expect_tx(full, C::kTileBytes);
         if constexpr (kPaged) {
           // keys row .. row+127 of sequence s live in eight 16-token pages; pages past the
           // sequence's end (masked by the softmax) read as zeros through an out-of-range block
@@ -458,14 +458,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           for (int r = 0; r < kBN / 16; ++r)
             for (int ch = 0; ch < C::kChunks; ++ch)
               tma_load_4d(sKV + st * C::kTileBytes + ch * C::kChunkBytes + r * 16 * 128, map,
-                          &kv_full[st], ch * 64, 0, h, blk[r]);
+                          full, ch * 64, 0, h, blk[r]);
         } else {
           for (int ch = 0; ch < C::kChunks; ++ch)
-            tma_load_3d(sKV + st * C::kTileBytes + ch * C::kChunkBytes, map, &kv_full[st], ch * 64,
-                        row, bh);
+            tma_load_3d(sKV + st * C::kTileBytes + ch * C::kChunkBytes, map, full, ch * 64, row,
+                        bh);
         }
-        issued[st] = true;
-        last_ph[st] = ph;
+        ++loads[(is_v ? C::kStages : 0) + st];
         ++kv_it;
         return true;
       };
@@ -490,35 +489,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tma_load_3d(sQ + i * C::kTileBytes + ch * C::kChunkBytes, &tm_q, q_full, ch * 64,
                         (kGeneral ? p.q_row0 : 0) + pr * 2 * kBM + i * kBM, w.bh);
         }
-        if (!load_kv(&tm_k, 0, w.bh)) { ok = false; break; }
+        if (!load_kv(&tm_k, 0, w.bh, false)) { ok = false; break; }
         for (int j = 0; ok && j < nmax; ++j) {
-          if (j + 1 < nmax && !load_kv(&tm_k, (j + 1) * kBN, w.bh)) { ok = false; break; }
-          if (!load_kv(&tm_v, j * kBN, w.bh)) { ok = false; break; }
+          if (j + 1 < nmax && !load_kv(&tm_k, (j + 1) * kBN, w.bh, false)) { ok = false; break; }
+          if (!load_kv(&tm_v, j * kBN, w.bh, true)) { ok = false; break; }
         }
       }
       if (!ok) {
         // abandoned: let every copy already in flight land before the CTA's smem goes away
         volatile int never = 0;
-        for (int s = 0; s < C::kStages; ++s)
-          if (issued[s]) mbar_wait(&kv_full[s], last_ph[s], &never);
+        for (int b = 0; b < 2 * C::kStages; ++b)
+          if (loads[b] > 0) mbar_wait(&kv_full[b], (loads[b] - 1) & 1, &never);
         if (q_issued) mbar_wait(q_full, q_ph ^ 1, &never);
       }
     }
-  } else if (C::kTwoIssuers && (warp == 9 || warp == 10)) {
+  } else if (warp == 9 || warp == 10) {
     // ------------------------------------------------------------------ MMA issuers (two)
     // Warp 9 issues S_i,j = Q_i K_j^T, warp 10 issues O_i += P_i,j V_j, each in block order and
     // each committing its own barriers; K_j's stage is released by the first, V_j's by the second.
     // Per unit the loads arrive in the order K_0, then K_{j+1}, V_j for j = 0, 1, ...: load index
-    // of K_j is 2j-1 (K_0: 0), of V_j 2j+2 (2j+1 for the last block).  A stage is reloaded only
-    // after the issuer that waits on its previous load has released it, so a parity wait can never
-    // see a phase two steps ahead.
+    // of K_j is 2j-1 (K_0: 0), of V_j 2j+2 (2j+1 for the last block).
     if (lane == 0) {
       const bool scores = warp == 9;
       uint32_t kv_base = 0, q_ph = 0;
       uint32_t s_cnt[2] = {0, 0};  // S_i computed so far (s_free phases follow it)
       uint32_t p_cnt[2] = {0, 0};  // P_i consumed so far (p_full phases follow it)
+      uint32_t full_ph = 0;        // bit st: phase parity of this issuer's landing barrier of stage st
       const uint32_t sQ0 = smem_u32(sQ), sQ1 = smem_u32(sQ + C::kTileBytes);
       const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
+      uint64_t *my_full = kv_full + (scores ? 0 : C::kStages);
+      auto wait_load = [&](uint32_t st) -> bool {
+        if (!mbar_wait(&my_full[st], (full_ph >> st) & 1u, abort_flag)) return false;
+        full_ph ^= 1u << st;
+        return true;
+      };
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int u = unit_for_round<kGeneral>(p, r, seq_order);
@@ -533,7 +537,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           for (int j = 0; ok && j < nmax; ++j) {
             const uint32_t ld = kv_base + (j == 0 ? 0u : static_cast<uint32_t>(2 * j - 1));
             const uint32_t st = ld % C::kStages;
-            if (!mbar_wait(&kv_full[st], (ld / C::kStages) & 1, abort_flag)) { ok = false; break; }
+            if (!wait_load(st)) { ok = false; break; }
             for (int i = 0; i < 2; ++i) {
               if (j >= n[i]) continue;
               if (s_cnt[i] > 0 && !mbar_wait(&s_free[i], (s_cnt[i] - 1) & 1, abort_flag)) {
@@ -555,7 +559,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           for (int j = 0; ok && j < nmax; ++j) {
             const uint32_t ld = kv_base + static_cast<uint32_t>(j + 1 < nmax ? 2 * j + 2 : 2 * j + 1);
             const uint32_t st = ld % C::kStages;
-            if (!mbar_wait(&kv_full[st], (ld / C::kStages) & 1, abort_flag)) { ok = false; break; }
+            if (!wait_load(st)) { ok = false; break; }
             for (int i = 0; i < 2; ++i) {
               if (j >= n[i]) continue;
               if (!mbar_wait(&p_full[i], p_cnt[i] & 1, abort_flag)) { ok = false; break; }
@@ -577,178 +581,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       umma_commit(&drain[scores ? 0 : 1]);
       volatile int never = 0;
       mbar_wait(&drain[scores ? 0 : 1], 0, &never);
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
-    if constexpr (C::kEventMma) {
-      // Event-driven: each pass polls (without blocking) what each tile can take next -- S_i,j once
-      // K_j has landed and the softmax has copied out S_i,j-1, or O_i += P_i,j V_j once V_j has
-      // landed and P_i,j is written -- and issues whatever is ready, scores first, so that neither
-      // tile's softmax waits behind the other tile's work.  Per unit the loads arrive in the order
-      // K_0, then K_{j+1}, V_j for j = 0, 1, ...: load index of K_j is 2j-1 (K_0: 0), of V_j 2j+2
-      // (2j+1 for the last block, which has no K_{j+1} before it).  A load is only tested once the
-      // earlier load that used its stage has landed (its consumer was issued first), so the parity
-      // test cannot see a stale phase.
-      if (lane == 0) {
-        uint32_t kv_base = 0, q_ph = 0;
-        uint32_t s_cnt[2] = {0, 0};  // S_i computed so far (s_free phases follow it)
-        uint32_t p_cnt[2] = {0, 0};  // P_i consumed so far (p_full phases follow it)
-        const uint32_t sQ0 = smem_u32(sQ), sQ1 = smem_u32(sQ + C::kTileBytes);
-        const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
-        bool ok = true;
-        for (int r = 0; ok; ++r) {
-          const int u = unit_for_round<kGeneral>(p, r, seq_order);
-          if (u < 0) break;
-          const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
-          const int pr = w.pair;
-          const KvSpan kv = kv_span<kMode>(p, w.bh);
-          const int n[2] = {tile_blocks(p, kv, pr, 0), tile_blocks(p, kv, pr, 1)};
-          const int nmax = n[0] > n[1] ? n[0] : n[1];
-          if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
-          q_ph ^= 1;
-          tc_fence_after();
-          int s_next[2] = {0, 0}, pv_next[2] = {0, 0};
-          int s_left = n[0] + n[1], pv_left = n[0] + n[1];
-          auto k_load = [&](int j) { return kv_base + (j == 0 ? 0u : static_cast<uint32_t>(2 * j - 1)); };
-          auto v_load = [&](int j) {
-            return kv_base + static_cast<uint32_t>(j + 1 < nmax ? 2 * j + 2 : 2 * j + 1);
-          };
-          auto landed = [&](uint32_t ld) {
-            return mbar_test(&kv_full[ld % C::kStages], (ld / C::kStages) & 1);
-          };
-          uint64_t t_last = globaltimer_ns();
-          while (pv_left > 0) {
-            bool progressed = false;
-            for (int i = 0; i < 2; ++i) {
-              const int j = s_next[i];
-              if (j >= n[i]) continue;
-              const uint32_t kld = k_load(j);
-              if (!landed(kld)) continue;
-              if (s_cnt[i] > 0 && !mbar_test(&s_free[i], (s_cnt[i] - 1) & 1)) continue;
-              tc_fence_after();
-              issue_qk<HD>(tmem + (i ? C::kColS1 : C::kColS0), i ? sQ1 : sQ0,
-                           sKV0 + (kld % C::kStages) * C::kTileBytes);
-              umma_commit(&s_full[i]);
-              ++s_cnt[i];
-              ++s_next[i];
-              --s_left;
-              progressed = true;
-              // K_j is free once every tile that visits block j has computed its S_i,j
-              const int other = s_next[i ^ 1];
-              if (j >= n[i ^ 1] || other > j) umma_commit(&kv_empty[kld % C::kStages]);
-              if (s_left == 0) umma_commit(q_empty);  // every Q K^T of the unit is issued
-            }
-            for (int i = 0; i < 2; ++i) {
-              const int j = pv_next[i];
-              if (j >= n[i] || j >= s_next[i]) continue;
-              const uint32_t vld = v_load(j);
-              if (!landed(vld)) continue;
-              if (!mbar_test(&p_full[i], p_cnt[i] & 1)) continue;
-              ++p_cnt[i];
-              tc_fence_after();
-              const uint32_t p_addr = C::kPInTmem ? tmem + (i ? C::kColP1 : C::kColP0)
-                                                  : sP0 + i * C::kPBytes;
-              issue_pv<HD>(tmem + (i ? C::kColO1 : C::kColO0), p_addr,
-                           sKV0 + (vld % C::kStages) * C::kTileBytes, j > 0);
-              umma_commit(&pv_done[i]);
-              ++pv_next[i];
-              --pv_left;
-              progressed = true;
-              const int other = pv_next[i ^ 1];
-              if (j >= n[i ^ 1] || other > j) umma_commit(&kv_empty[vld % C::kStages]);
-            }
-            if (progressed) {
-              t_last = globaltimer_ns();
-            } else {
-              if (*abort_flag) { ok = false; break; }
-              if (globaltimer_ns() - t_last > FA_WAIT_LIMIT_NS) {
-                *abort_flag = 1;
-                atomicExch(&g_device_status, 5 /* FA_ERR_TIMEOUT */);
-                ok = false;
-                break;
-              }
-            }
-          }
-          kv_base += 2 * nmax;
-        }
-        // every MMA issued by this thread completes before TMEM is released
-        umma_commit(&drain[0]);
-        volatile int never = 0;
-        mbar_wait(&drain[0], 0, &never);
-      }
-    } else {
-      if (lane == 0) {
-        uint32_t kv_it = 0, q_ph = 0;
-        uint32_t s_cnt[2] = {0, 0};  // S_i computed so far (s_free phases follow it)
-        uint32_t p_cnt[2] = {0, 0};  // P_i consumed so far
-        const uint32_t sQ0 = smem_u32(sQ), sQ1 = smem_u32(sQ + C::kTileBytes);
-        const uint32_t sKV0 = smem_u32(sKV), sP0 = smem_u32(sP);
-        bool ok = true;
-        // S_i = Q_i K^T into S_i's TMEM columns, once the softmax has copied out the previous S_i.
-        auto issue_s = [&](int i, uint32_t k_stage) -> bool {
-          if (s_cnt[i] > 0 && !mbar_wait(&s_free[i], (s_cnt[i] - 1) & 1, abort_flag)) return false;
-          tc_fence_after();
-          issue_qk<HD>(tmem + (i ? C::kColS1 : C::kColS0), i ? sQ1 : sQ0,
-                       sKV0 + k_stage * C::kTileBytes);
-          umma_commit(&s_full[i]);
-          ++s_cnt[i];
-          return true;
-        };
-        for (int r = 0; ok; ++r) {
-          const int u = unit_for_round<kGeneral>(p, r, seq_order);
-          if (u < 0) break;
-          const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
-          const int pr = w.pair;
-          const KvSpan kv = kv_span<kMode>(p, w.bh);
-          const int n[2] = {tile_blocks(p, kv, pr, 0), tile_blocks(p, kv, pr, 1)};
-          const int nmax = n[0] > n[1] ? n[0] : n[1];
-          if (!mbar_wait(q_full, q_ph, abort_flag)) { ok = false; break; }
-          q_ph ^= 1;
-          {
-            const uint32_t st = kv_it % C::kStages, ph = (kv_it / C::kStages) & 1;
-            if (!mbar_wait(&kv_full[st], ph, abort_flag)) { ok = false; break; }
-            for (int i = 0; ok && i < 2; ++i)
-              if (n[i] > 0 && !issue_s(i, st)) ok = false;
-            if (!ok) break;
-            umma_commit(&kv_empty[st]);  // K_0 is free once both S_i,0 have been computed
-            ++kv_it;
-            if (nmax == 1) umma_commit(q_empty);
-          }
-          for (int j = 0; ok && j < nmax; ++j) {
-            if (j + 1 < nmax) {
-              // the next scores first: they only need K_{j+1} and the softmax's copy of S_i,j
-              const uint32_t st = kv_it % C::kStages, ph = (kv_it / C::kStages) & 1;
-              if (!mbar_wait(&kv_full[st], ph, abort_flag)) { ok = false; break; }
-              for (int i = 0; ok && i < 2; ++i)
-                if (j + 1 < n[i] && !issue_s(i, st)) ok = false;
-              if (!ok) break;
-              umma_commit(&kv_empty[st]);
-              ++kv_it;
-              if (j + 2 == nmax) umma_commit(q_empty);  // that was the last Q K^T of the unit
-            }
-            const uint32_t vst = kv_it % C::kStages, vph = (kv_it / C::kStages) & 1;
-            if (!mbar_wait(&kv_full[vst], vph, abort_flag)) { ok = false; break; }
-            for (int i = 0; ok && i < 2; ++i) {
-              if (j >= n[i]) continue;
-              if (!mbar_wait(&p_full[i], p_cnt[i] & 1, abort_flag)) { ok = false; break; }
-              ++p_cnt[i];
-              tc_fence_after();
-              const uint32_t p_addr = C::kPInTmem ? tmem + (i ? C::kColP1 : C::kColP0)
-                                                  : sP0 + i * C::kPBytes;
-              issue_pv<HD>(tmem + (i ? C::kColO1 : C::kColO0), p_addr, sKV0 + vst * C::kTileBytes,
-                           j > 0);
-              umma_commit(&pv_done[i]);
-            }
-            if (!ok) break;
-            umma_commit(&kv_empty[vst]);
-            ++kv_it;
-          }
-        }
-        // every MMA issued by this thread completes before TMEM is released
-        umma_commit(&drain[0]);
-        volatile int never = 0;
-        mbar_wait(&drain[0], 0, &never);
-      }
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax / epilogue
@@ -786,18 +618,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int pr = w.pair;
       const KvSpan kv = kv_span<kMode>(p, w.bh);
       const int n = tile_blocks(p, kv, pr, wg);
+      // no turns in a unit with one tile only (a ragged last pair, a draft tree of <= 128 nodes):
+      // both warps of a pair see the same block counts, so they skip the same units
       const int n_other = tile_blocks(p, kv, pr, wg ^ 1);
-      if (n == 0) {
-        // a tile past the last query row: only its turns
-        if constexpr (C::kExpTurns) {
-          for (int j = 0; ok && j < n_other; ++j) {
-            if (!take_turn()) ok = false;
-            else pass_turn();
-          }
-        }
-        if (!ok) break;
-        continue;
-      }
+      const bool turns = C::kExpTurns && n > 0 && n_other > 0;
+      if (n == 0) continue;
       const int qrow = pr * 2 * kBM + wg * kBM + row;
       const bool tree = kPaged && p.tree_mask != nullptr;
       const uint64_t tmask =
@@ -861,10 +686,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
         uint32_t pk[kBN / 2];
-        if (C::kExpTurns && !take_turn()) { ok = false; break; }
+        if (turns && !take_turn()) { ok = false; break; }
         const float p_top = ex2(fmaf(s_top, sl2, mneg));
-        const float le = FA_EXP_SCHEDULE ? exp_row_pipelined(s, sl2, mneg, pk) : exp_row(s, sl2, mneg, pk);
-        if (C::kExpTurns) pass_turn();
+        const float le = FA_EXP_SCHEDULE ? exp_row_pipelined(s, sl2, mneg, pk) : exp_row<kPolyEvery<HD>>(s, sl2, mneg, pk);
+        if (turns) pass_turn();
         // O is normalised by the sum of the bf16-rounded p that P V uses, so that it is a
         // convex combination of V rows even when one key dominates the row; the rounding error
         // that matters is the largest element's, so the fp32 sum is corrected by exactly that
@@ -914,7 +739,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[wg]);  // one arrival per warp
       }
-      if (C::kExpTurns) {
+      if (turns) {
         // the other tile's extra block (causal pairs: tile 1 has one more)
         for (int j = n; ok && j < n_other; ++j) {
           if (!take_turn()) ok = false;
