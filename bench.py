@@ -513,6 +513,15 @@ def bench_ours(args, rank, world):
     if args.only == "paged":
         return {"metric": METRIC,
                 "paged_prefill": bench_paged_prefill(fa, args, dev, flush, stream, pk)}
+    if args.only == "point":
+        # one sweep point alone (for profiling): d, N and the mask from the command line
+        case = next(c for c in W.sweep_cases(args.point_d)
+                    if c.N == args.point_n and c.causal == bool(args.point_causal))
+        ts = run_prefill_case(fa, case, args.steps, args.warmup, flush, stream)
+        ms = statistics.median(ts)
+        return {"metric": METRIC, "point": {"d": case.d, "N": case.N, "B": case.B, "H": case.H,
+                                            "causal": case.causal, "ms": round(ms, 4),
+                                            "tflops": round(case.flops / (ms * 1e-3) / 1e12, 1)}}
 
     # ---- headline: prefill config, non-causal + causal per step
     cases = W.prefill_cases()
@@ -745,8 +754,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="sequences in the decode workload (64 is the benchmark; fewer for profiling)")
+    ap.add_argument("--point-d", type=int, default=64, help="--only point: head dim")
+    ap.add_argument("--point-n", type=int, default=4096, help="--only point: sequence length")
+    ap.add_argument("--point-causal", type=int, default=0, help="--only point: causal (0/1)")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "paged", "backward", "tree",
-                                       "seqpar"],
+                                       "seqpar", "point"],
                     default="all",
                     help="prefill: the headline loop alone; decode / paged: the paged decode or "
                     "chunked prefill loop alone")
