@@ -49,9 +49,9 @@ constexpr int kPrefillThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale: tolerate a stale max up to 2^8 below
 constexpr float kLn2 = 0.6931471805599453f;
 // every kPolyEvery-th pair of P's exponentials is evaluated on the FMA pipe, the rest on MUFU
-// (0: all MUFU).  At d = 128 every share tried (1/8 .. 1/2) was slower; at d = 64 a quarter was
-// about 7% faster but pushed peaked rows past the parity bound (max|dO| 1.25e-2 at N = 16k), so
-// both head dims use MUFU only.
+// (0: all MUFU).  Measured on the B200: at d = 128 every share tried (1/8 .. 1/2) was slower; at
+// d = 64 a quarter was 14-20% slower once the normaliser sums the rounded values exactly (which
+// the polynomial share needs for parity on rows dominated by one key).  So MUFU only.
 #ifndef FA_POLY_EVERY
 #define FA_POLY_EVERY 0
 #endif
@@ -67,9 +67,11 @@ struct PrefillCfg {
   static constexpr int kChunks = HD / 64;          // 64-element (128-byte) swizzle chunks per row
   static constexpr int kChunkBytes = 128 * 128;    // 128 rows x 128 bytes
   static constexpr int kTileBytes = 128 * HD * 2;  // one 128 x HD bf16 tile
-  // P lives in TMEM when there is room for it beside S and O (d = 64: S 2x128 + O 2x64 + P 2x64
-  // columns = 512), otherwise in shared memory (d = 128: S and O fill all 512 columns).
-  static constexpr bool kPInTmem = HD == 64;
+  // P is staged in shared memory at both head dims.  At d = 64 it would also fit in TMEM beside S
+  // and O (S 2x128 + O 2x64 + P 2x64 columns = 512), and P V could read it from there, but the
+  // asynchronous tcgen05.st of P keeps its 64 registers allocated longer and the instance spilled;
+  // staged in shared memory it does not, and measured 4-6% faster.  kPInTmem keeps both paths.
+  static constexpr bool kPInTmem = false;
   // Exponential turns: softmax warp w (tile 0) and warp w + 4 (tile 1) run on the same SM
   // sub-partition and share its special-function unit, which evaluates a row block's 128
   // exponentials per thread about as fast as the tensor core does the block's MMAs.  Left to
@@ -250,11 +252,14 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_addr, uint3
 // One row of a score block -> P: p = 2^(s * scale*log2e - m_ref) for the 128 scores of this
 // thread's row (MUFU ex2, or the FMA-pipe polynomial for every kPolyEvery-th pair), packed to
 // bf16 pairs in pk.  Returns the sum of the fp32 p.
+// With kPoly > 0 it also returns in `rounded` the exact sum of the bf16 values in pk (the P that
+// P V uses): the polynomial and MUFU round differently, so the single-element correction the
+// MUFU-only path uses (below) would not match the element actually stored.
 template <int kPoly>
 __device__ __forceinline__ float exp_row(float (&s)[kBN], float sl2, float mneg,
-                                         uint32_t (&pk)[kBN / 2]) {
+                                         uint32_t (&pk)[kBN / 2], float &rounded) {
   const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(mneg, mneg);
-  uint64_t le2 = 0;
+  uint64_t le2 = 0, lr2 = 0;
 #pragma unroll
   for (int c = 0; c < kBN / 2; ++c) {
     const uint64_t x2 = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), c2, m2);
@@ -270,42 +275,15 @@ __device__ __forceinline__ float exp_row(float (&s)[kBN], float sl2, float mneg,
     float p0, p1;
     f2_unpack(p2, p0, p1);
     pk[c] = pack_bf16x2(p0, p1);
+    if constexpr (kPoly > 0)
+      lr2 = f2_add(lr2, f2_pack(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xffff0000u)));
   }
   float a, b;
+  if constexpr (kPoly > 0) {
+    f2_unpack(lr2, a, b);
+    rounded = a + b;
+  }
   f2_unpack(le2, a, b);
-  return a + b;
-}
-
-#ifndef FA_EXP_SCHEDULE
-#define FA_EXP_SCHEDULE 0
-#endif
-#ifndef FA_EXP_LOOKAHEAD
-#define FA_EXP_LOOKAHEAD 4
-#endif
-
-// Same contract as exp_row, written so that in-order issue keeps MUFU busy: every score is first
-// scaled and shifted in place, then each step issues the exponentials FA_EXP_LOOKAHEAD pairs ahead
-// of the pair it packs and sums (schedule 2), or all exponentials before any packing (schedule 1).
-__device__ __forceinline__ float exp_row_pipelined(float (&s)[kBN], float sl2, float mneg,
-                                                   uint32_t (&pk)[kBN / 2]) {
-  const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(mneg, mneg);
-#pragma unroll
-  for (int e = 0; e < kBN; e += 2) f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, m2), s[e], s[e + 1]);
-  constexpr int L = FA_EXP_SCHEDULE == 1 ? kBN / 2 : FA_EXP_LOOKAHEAD;
-#pragma unroll
-  for (int e = 0; e < 2 * L; ++e) s[e] = ex2(s[e]);
-  uint64_t a2 = 0;
-#pragma unroll
-  for (int c = 0; c < kBN / 2; ++c) {
-    if (c + L < kBN / 2) {
-      s[2 * (c + L)] = ex2(s[2 * (c + L)]);
-      s[2 * (c + L) + 1] = ex2(s[2 * (c + L) + 1]);
-    }
-    a2 = f2_add(a2, f2_pack(s[2 * c], s[2 * c + 1]));
-    pk[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
-  }
-  float a, b;
-  f2_unpack(a2, a, b);
   return a + b;
 }
 
@@ -687,16 +665,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
         uint32_t pk[kBN / 2];
         if (turns && !take_turn()) { ok = false; break; }
-        const float p_top = ex2(fmaf(s_top, sl2, mneg));
-        const float le = FA_EXP_SCHEDULE ? exp_row_pipelined(s, sl2, mneg, pk) : exp_row<kPolyEvery<HD>>(s, sl2, mneg, pk);
+        constexpr int kPoly = kPolyEvery<HD>;
+        float lr_blk = 0.f;
+        const float p_top = kPoly > 0 ? 0.f : ex2(fmaf(s_top, sl2, mneg));
+        const float le = exp_row<kPoly>(s, sl2, mneg, pk, lr_blk);
         if (turns) pass_turn();
         // O is normalised by the sum of the bf16-rounded p that P V uses, so that it is a
-        // convex combination of V rows even when one key dominates the row; the rounding error
-        // that matters is the largest element's, so the fp32 sum is corrected by exactly that
-        // element's rounding (same arithmetic as in exp_row).  The LSE keeps the fp32 sum.
-        const float p_top_r = __uint_as_float(pack_bf16x2(0.f, p_top) & 0xffff0000u);
+        // convex combination of V rows even when one key dominates the row.  With MUFU only, the
+        // rounding error that matters is the largest element's, so the fp32 sum is corrected by
+        // exactly that element's rounding (same arithmetic as in exp_row); with the polynomial
+        // share, exp_row sums the rounded values themselves.  The LSE keeps the fp32 sum.
+        if constexpr (kPoly == 0)
+          lr_blk = le + (__uint_as_float(pack_bf16x2(0.f, p_top) & 0xffff0000u) - p_top);
         l = l * alpha + le;
-        lr = lr * alpha + le + (p_top_r - p_top);
+        lr = lr * alpha + lr_blk;
         if (j > 0) {
           // P_i,j-1 must have been consumed (and O_i completed through block j-1) before this
           // block's P overwrites the smem tile and before O_i is rescaled
@@ -704,10 +686,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           pv_ph ^= 1;
           tc_fence_after();
         }
-        // P first: its registers are free before O's rescale
+        // P first, then O's rescale.  A tcgen05.st reads its source registers asynchronously, so
+        // they stay allocated until tcgen05.wait::st: wait right after each store, so that P's 64
+        // registers and each rescaled chunk of O are free again before the next use (waiting only
+        // once at the end held them all at once and made the d = 64 instance spill).
         if constexpr (C::kPInTmem) {
           tmem_st32(tP, pk);
           tmem_st32(tP + 32, pk + 32);
+          tmem_wait_st();
         } else {
           if (kTmaO && !C::kPInTmem && p.o_tma && j == 0) {
             // the previous unit's O left this warp's rows of the P tile through tensor stores
@@ -727,14 +713,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
               tmem_st32(tO + cc, o);
+              tmem_wait_st();
             }
           }
         }
-        if constexpr (C::kPInTmem) tmem_wait_st();
-        else {
-          tmem_wait_st();
-          fence_async_smem();  // generic-proxy smem writes -> visible to the tensor core
-        }  // generic-proxy smem writes -> visible to the tensor core
+        if constexpr (!C::kPInTmem) fence_async_smem();  // generic-proxy P -> the tensor core
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[wg]);  // one arrival per warp
