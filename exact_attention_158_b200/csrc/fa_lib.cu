@@ -190,6 +190,42 @@ bool encode_pool(CUtensorMap *map, const void *base, int d, int H, int num_block
   return r == CUDA_SUCCESS;
 }
 
+// The d = 128 V pool as a 5-D tensor (64 columns, 16 tokens, 2 column halves, H, num_blocks) read
+// in 64 x 16 x 2 x 1 x 1 boxes: a whole 16-token page of one head (4 KB) per load, landing as
+// [half][token][64 columns].  The half stride (128 bytes) is smaller than the token stride (256
+// bytes): the box reorders the page so that each half is the 16 x 128-byte K-group pair the P V
+// product reads for its 16 keys.
+// The d = 128 K pool as a 5-D tensor (64 columns, 8 tokens, 2 column chunks, 2 token groups,
+// num_blocks * H pages of one head) read in 64 x 8 x 2 x 2 x 1 boxes: a whole 16-token page of one
+// head (4 KB) per load, landing as [token group][chunk][8 tokens][64 columns].  Eight such pages
+// make a K tile whose 8-key groups (1 KB swizzle atoms) sit 2 KB apart for each 64-column chunk,
+// the layout issue_qk reads for the paged mode.
+bool encode_pool_k_pages(CUtensorMap *map, const void *base, int H, int num_blocks) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[5] = {64, 8, 2, 2, static_cast<cuuint64_t>(num_blocks) * H};
+  cuuint64_t strides[4] = {256, 128, 8 * 256, 16 * 256};
+  cuuint32_t box[5] = {64, 8, 2, 2, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_pool_v_pages(CUtensorMap *map, const void *base, int H, int num_blocks) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[5] = {64, 16, 2, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(num_blocks)};
+  cuuint64_t strides[4] = {256, 128, 16 * 256, static_cast<cuuint64_t>(H) * 16 * 256};
+  cuuint32_t box[5] = {64, 16, 2, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int HD, int kMode>
 fa_status launch_prefill(DeviceInfo &dev, const CUtensorMap &tq, const CUtensorMap &tk,
                          const CUtensorMap &tv, fa::PrefillParams p, cudaStream_t stream,
@@ -593,6 +629,8 @@ static fa_status prefill_paged_impl(const void *q, const void *k_pool, const voi
   if (static_cast<long long>(S) * H * Lq > INT_MAX) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(max_blocks_per_seq) * fa::kPage > INT_MAX) return FA_ERR_INVALID_ARG;
   if (Lq > max_blocks_per_seq * fa::kPage) return FA_ERR_INVALID_ARG;
+  // the d = 128 K map indexes (block, head) pages as block * H + head, block up to num_blocks
+  if ((static_cast<long long>(num_blocks) + 1) * H > INT_MAX) return FA_ERR_INVALID_ARG;
   float sc;
   if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o))
@@ -615,8 +653,13 @@ static fa_status prefill_paged_impl(const void *q, const void *k_pool, const voi
   if (st != FA_OK) return st;
   CUtensorMap tq, tk, tv;
   const int BH = S * H;
-  if (!encode_bhnd(&tq, q, d, Lq, BH) || !encode_pool(&tk, k_pool, d, H, num_blocks) ||
-      !encode_pool(&tv, v_pool, d, H, num_blocks)) {
+  // d = 128: K and V pages arrive as one 4 KB box each (see encode_pool_k_pages / _v_pages)
+  const bool pages = d == 128;
+  if (!encode_bhnd(&tq, q, d, Lq, BH) ||
+      !(pages ? encode_pool_k_pages(&tk, k_pool, H, num_blocks)
+              : encode_pool(&tk, k_pool, d, H, num_blocks)) ||
+      !(pages ? encode_pool_v_pages(&tv, v_pool, H, num_blocks)
+              : encode_pool(&tv, v_pool, d, H, num_blocks))) {
     t_last_error = "cuTensorMapEncodeTiled failed";
     return FA_ERR_LAUNCH;
   }

@@ -216,14 +216,20 @@ __device__ __forceinline__ int tile_blocks(const PrefillParams &p, const KvSpan 
 // address below 2^18 (all of shared memory), desc(addr + off) = desc(addr) + off / 16 exactly.
 
 // S (TMEM) = Q (smem, K-major) K^T (smem, K-major), K = HD in steps of 16.
-template <int HD>
+// K tile layouts: [64-column chunk][128 keys][128 B] (8-key atoms 1 KB apart, chunks kChunkBytes
+// apart), or with kPageKV (paged mode, d = 128: one 4 KB load per 16-token page)
+// [page][8-key group][chunk][8 keys][128 B]: 8-key atoms 2 KB apart, chunk 1 at +1 KB.
+template <int HD, bool kPageKV = false>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
   using C = PrefillCfg<HD>;
-  const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024), kd = smem_desc_sw128(k_smem, 16, 1024);
+  constexpr uint32_t kKChunk = kPageKV ? 1024 : C::kChunkBytes;
+  const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024);
+  const uint64_t kd = smem_desc_sw128(k_smem, 16, kPageKV ? 2048 : 1024);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
-    const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kChunkBytes + (kk % 4) * 32) >> 4);
-    umma_ss(d_tmem, qd + off, kd + off, C::kIdescQK, kk > 0 ? 1u : 0u);
+    const uint64_t qoff = static_cast<uint64_t>(((kk / 4) * C::kChunkBytes + (kk % 4) * 32) >> 4);
+    const uint64_t koff = static_cast<uint64_t>(((kk / 4) * kKChunk + (kk % 4) * 32) >> 4);
+    umma_ss(d_tmem, qd + qoff, kd + koff, C::kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -231,15 +237,19 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint3
 // 16.  V's descriptor: LBO = distance between 64-element chunks of d, SBO = between 8-key groups.
 // p_addr is a shared-memory address, or with kPInTmem a TMEM address (2 bf16 per column, 8
 // columns per 16 keys).
-template <int HD>
+// V tile layouts: [64-column chunk][128 keys][128 B] (chunks kChunkBytes apart), or with kPageKV
+// (paged mode, d = 128: one 4 KB load per 16-token page) [page][64-column half][16 keys][128 B],
+// a page per 16-key step and its halves 2 KB apart.
+template <int HD, bool kPageKV = false>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_addr, uint32_t v_smem,
                                          bool accumulate) {
   using C = PrefillCfg<HD>;
-  const uint64_t vd = smem_desc_sw128(v_smem, C::kChunkBytes, 1024);
+  constexpr uint32_t kStepBytes = kPageKV ? 4096 : 16 * 128;  // V bytes per 16-key step
+  const uint64_t vd = smem_desc_sw128(v_smem, kPageKV ? 2048 : C::kChunkBytes, 1024);
   const uint64_t pd = C::kPInTmem ? 0 : smem_desc_sw128(p_addr, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk) {
-    const uint64_t b = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
+    const uint64_t b = vd + static_cast<uint64_t>((kk * kStepBytes) >> 4);
     if constexpr (C::kPInTmem) {
       umma_ts(o_tmem, p_addr + kk * 8, b, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
     } else {
@@ -314,6 +324,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   using C = PrefillCfg<HD>;
   constexpr bool kPaged = kMode == kModePaged;
   constexpr bool kGeneral = kMode != kModeSquare;  // key count and query offset per unit
+  constexpr bool kPageKV = kPaged && HD == 128;     // K and V pages arrive as whole 4 KB boxes
   // bf16 O through a shared-memory staging tile and tensor stores (square and paged modes: the
   // processed rows of (b, h) are rows 0 .. N-1 of its O slice)
   constexpr bool kTmaO = kMode != kModeRange;
@@ -432,11 +443,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             blk[r] = b;
           }
+          if (kPageKV) {
+            // d = 128: one 4 KB box per page (the layouts issue_qk and issue_pv read with
+            // kPageKV): a TMA box costs about as much fixed time as 10 KB of data, so eight boxes
+            // per tile instead of sixteen.  K's map indexes pages of one head as block * H + head
+            // (an out-of-range block stays out of range), V's as (head, block).
 #pragma unroll
-          for (int r = 0; r < kBN / 16; ++r)
-            for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_load_4d(sKV + st * C::kTileBytes + ch * C::kChunkBytes + r * 16 * 128, map,
-                          full, ch * 64, 0, h, blk[r]);
+            for (int r = 0; r < kBN / 16; ++r) {
+              if (is_v)
+                tma_load_5d(sKV + st * C::kTileBytes + r * 4096, map, full, 0, 0, 0, h, blk[r]);
+              else
+                tma_load_5d(sKV + st * C::kTileBytes + r * 4096, map, full, 0, 0, 0, 0,
+                            blk[r] * p.H + h);
+            }
+          } else {
+#pragma unroll
+            for (int r = 0; r < kBN / 16; ++r)
+              for (int ch = 0; ch < C::kChunks; ++ch)
+                tma_load_4d(sKV + st * C::kTileBytes + ch * C::kChunkBytes + r * 16 * 128, map,
+                            full, ch * 64, 0, h, blk[r]);
+          }
         } else {
           for (int ch = 0; ch < C::kChunks; ++ch)
             tma_load_3d(sKV + st * C::kTileBytes + ch * C::kChunkBytes, map, full, ch * 64, row,
@@ -523,8 +549,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 break;
               }
               tc_fence_after();
-              issue_qk<HD>(tmem + (i ? C::kColS1 : C::kColS0), i ? sQ1 : sQ0,
-                           sKV0 + st * C::kTileBytes);
+              issue_qk<HD, kPageKV>(tmem + (i ? C::kColS1 : C::kColS0), i ? sQ1 : sQ0,
+                                    sKV0 + st * C::kTileBytes);
               umma_commit(&s_full[i]);
               ++s_cnt[i];
             }
@@ -545,8 +571,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               tc_fence_after();
               const uint32_t p_addr = C::kPInTmem ? tmem + (i ? C::kColP1 : C::kColP0)
                                                   : sP0 + i * C::kPBytes;
-              issue_pv<HD>(tmem + (i ? C::kColO1 : C::kColO0), p_addr, sKV0 + st * C::kTileBytes,
-                           j > 0);
+              issue_pv<HD, kPageKV>(tmem + (i ? C::kColO1 : C::kColO0), p_addr,
+                                   sKV0 + st * C::kTileBytes, j > 0);
               umma_commit(&pv_done[i]);
             }
             if (!ok) break;

@@ -209,6 +209,7 @@ fa_status fa_decode_paged(const void *q, const void *k_pool, const void *v_pool,
  *                clamped into it and reported the same way).
  *   o            [S, H, Lq, d], bf16 or fp32 per o_dtype;  lse: fp32 [S, H, Lq] or NULL.
  *   S, H, Lq     >= 1, Lq <= 16 * max_blocks_per_seq;  d: 64 or 128;  causal 0/1;
+ *                (num_blocks + 1) * H <= INT_MAX (else FA_ERR_INVALID_ARG).
  *   scale        as for fa_fwd.
  * Returns FA_OK once the kernel is queued.  No workspace.
  */
