@@ -10,10 +10,12 @@
 //     dV_j = sum_i P_ij dO_i      dP_ij = dO_i . V_j      dS_ij = P_ij (dP_ij - D_i)
 //     dK_j = scale sum_i dS_ij Q_i                         dQ_i = scale sum_j dS_ij K_j
 //
-// Work partition: one CTA per (b, h, key block j of 128 keys).  K_j and V_j stay in shared memory;
-// the CTA streams every query block i that sees them (i >= j when causal) and keeps dK_j and dV_j
-// in TMEM for the whole loop.  dQ_i gets one 128 x d partial per (i, j) pair, added into an fp32
-// accumulator in global memory.
+// Work partition: a (b, h, key block j of 128 keys) sub-unit keeps K_j and V_j in shared memory,
+// streams every query block i that sees them (i >= j when causal) and keeps dK_j and dV_j in TMEM
+// for the whole loop.  dQ_i gets one 128 x d partial per (i, j) pair, added into an fp32
+// accumulator in global memory.  The kernel is persistent (at most one CTA per SM): each CTA
+// walks its sub-units in turn, so the next K_j, V_j and query blocks load, and the next block's
+// S^T and dP^T run on the tensor core, while the compute warps write the previous dK_j, dV_j.
 //
 // The scores are computed transposed, S^T = K_j Q_i^T (TMEM lane = key), so each compute thread
 // owns one key row: P^T and dS^T are written by rows into one 128 x 128 bf16 tile X in the
@@ -23,10 +25,11 @@
 // floats of one dQ row per warp instruction; at d = 64 it is dQ = dS K_j (lane = query).
 //
 //   warps 0-3, 4-7  compute, one key row per thread, query columns [0,64) and [64,128): P^T and
-//                   dS^T, and the final dK, dV write
+//                   dS^T, and each sub-unit's dK, dV write
 //   warps 8-11      dQ read-out: TMEM -> a shared-memory staging box -> a bulk tensor reduction
 //                   (fp32 add) into the accumulator, one box of 32 features per warp at a time
-//   warp  12        TMA producer: K_j, V_j once; Q_i (+ its LSE and D rows), dO_i per query block
+//   warp  12        TMA producer: K_j, V_j per sub-unit; Q_i (+ its LSE and D rows), dO_i per
+//                   query block
 //   warp  13        MMA issuer (one thread) + TMEM owner
 // TMEM (512 columns): S^T [0,128)  dP^T [128,256)  dV [256,256+d)  dK [256+d,256+2d); dQ at
 // [256+2d, 256+3d) when d = 64, and in S^T's columns when d = 128 (they are full otherwise).
@@ -60,7 +63,7 @@ struct BwdCfg {
   static constexpr bool kDqT = HD == 128;          // dQ^T in S^T's columns (lane = feature)
   static constexpr uint32_t kColDQ = kDqT ? kColS : 256 + 2 * HD;
   static constexpr int kTmemCols = 512;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 * kDoStages + 9;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 * kDoStages + 9;
   static constexpr size_t kBodyBytes = 2 * kTileBytes + (kStages + kDoStages) * kTileBytes +
                                        kXBytes + 4 * kStageSlotBytes + kStages * kVecFloats * 4 +
                                        kNumBars * 8 + 16;
@@ -82,7 +85,6 @@ struct BwdParams {
   float *dq_acc;      // [BH, Np, d] fp32, zero before the launch
   void *dk, *dv;      // [BH, N, d]
   int g_f32;          // dK / dV as fp32 (1) or bf16 (0)
-  int g_tma;          // d = 128, bf16 dK / dV: written by tensor stores (their maps were encoded)
   int BH, N, Np, nkb, causal;
   float scale_log2, scale;
 };
@@ -152,28 +154,6 @@ __device__ __forceinline__ void store_grad_cols(uint32_t taddr, int c0, float mu
         w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
         dst[e] = w;
       }
-    }
-  }
-}
-
-// d = 128, bf16 gradients: this thread's row (64 features from column c0 of TMEM, times mul) as
-// bf16 into row `lane` of a 32-row x 128-byte box, 128-byte swizzle (16-byte unit u at u ^ (r % 8)).
-__device__ __forceinline__ void stage_grad_box(uint32_t taddr, int c0, float mul, uint8_t *box,
-                                               int lane) {
-#pragma unroll
-  for (int ch = 0; ch < 2; ++ch) {
-    uint32_t v[32];
-    tmem_ld32(taddr + c0 + 32 * ch, v);
-    tmem_wait_ld();
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      uint4 w;
-      w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * mul, __uint_as_float(v[8 * e + 1]) * mul);
-      w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * mul, __uint_as_float(v[8 * e + 3]) * mul);
-      w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * mul, __uint_as_float(v[8 * e + 5]) * mul);
-      w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
-      const int u = ch * 4 + e;
-      *reinterpret_cast<uint4 *>(box + lane * 128 + ((u ^ (lane & 7)) * 16)) = w;
     }
   }
 }
@@ -257,8 +237,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_dq,
-                  const __grid_constant__ CUtensorMap tm_dk,
-                  const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
+                  const BwdParams p) {
   using C = BwdCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
@@ -289,24 +268,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t *dq_full = ds_full + 1;             // dK_i and dQ_i done: dQ_i readable, X free
   uint64_t *dq_free = dq_full + 1;             // dQ_i read out (4 warp arrivals)
   uint64_t *drain = dq_free + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *kv_empty = drain + 1;              // every product that reads K_j, V_j has completed
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(kv_empty + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int jb = blockIdx.x % p.nkb;  // key block
-  const int bh = blockIdx.x / p.nkb;
-  const int i_lo = p.causal ? jb : 0;  // first query block that sees key block jb
-  const int n = p.Np / kBM - i_lo;     // query blocks visited (>= 1)
-  // Visit order: step t takes query block i_lo + (t + rot) mod n.  The CTAs of one head run at the
-  // same time and all add into that head's dQ; starting each key block's loop at a different
-  // query block (rot = jb without the mask; with it, i_lo = jb already staggers them) keeps them
-  // from reducing into the same dQ rows at the same moment.
-  const int rot = p.causal ? 0 : jb % n;
-  auto qblock = [&](int t) { return i_lo + (t + rot) % n; };
+  // Persistent schedule.  The CTA takes pairs of key blocks (jb, nkb - 1 - jb) of one head, pair
+  // pu = blockIdx.x + m * gridDim.x (head-major), and processes the two as consecutive sub-units,
+  // the smaller jb first.  With the causal mask key block jb sees nkb - jb query blocks, so every
+  // pair costs the same nkb + 1 blocks and the round-robin deal is balanced; the CTAs running at
+  // the same time cover few heads, whose Q, dO and dQ rows stay in L2.
+  // sub_unit(k, bh, jb): 1 with (bh, jb) set, 0 once the CTA has no more, -1 for the empty second
+  // half of the middle pair (odd nkb).  Every role walks the same sequence.
+  const int npairs = (p.nkb + 1) / 2;
+  const int total_pairs = p.BH * npairs;
+  auto sub_unit = [&](int k, int &bh, int &jb) -> int {
+    const int pu = static_cast<int>(blockIdx.x) + (k / 2) * static_cast<int>(gridDim.x);
+    if (pu >= total_pairs) return 0;
+    bh = pu / npairs;
+    const int pp = pu % npairs;
+    jb = (k & 1) ? p.nkb - 1 - pp : pp;
+    return ((k & 1) && jb == pp) ? -1 : 1;
+  };
+  // Query blocks of key block jb (>= 1) and their visit order: step t takes query block
+  // i_lo + (t + rot) mod n.  Without the mask rot = jb staggers the key blocks of one head, so the
+  // CTAs adding into that head's dQ do not reduce into the same rows at the same moment (with it,
+  // i_lo = jb already staggers them).
+  struct Span {
+    int i_lo, n, rot;
+  };
+  auto span_of = [&](int jb) -> Span {
+    const int i_lo = p.causal ? jb : 0;
+    const int n = p.Np / kBM - i_lo;
+    return {i_lo, n, p.causal ? 0 : jb % n};
+  };
+  // Barrier phases run over the CTA's whole sequence of query blocks: block t of a sub-unit whose
+  // first block is the CTA's T-th has the global index T + t.
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
@@ -347,37 +349,64 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
-      int q_loads = 0, do_loads = 0;
-      mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
-      for (int ch = 0; ch < C::kChunks; ++ch) {
-        tma_load_3d(sK + ch * C::kChunkBytes, &tm_k, kv_full, ch * 64, jb * kBN, bh);
-        tma_load_3d(sV + ch * C::kChunkBytes, &tm_v, kv_full, ch * 64, jb * kBN, bh);
-      }
-      const size_t vec_row = static_cast<size_t>(bh) * p.Np;
-      for (int t = 0; t < n; ++t) {
-        const int i = qblock(t), st = t % C::kStages;
-        const uint32_t ph = (t / C::kStages) & 1;
-        if (!mbar_wait(&q_empty[st], ph ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&q_full[st], C::kTileBytes + C::kVecFloats * 4);
-        for (int ch = 0; ch < C::kChunks; ++ch)
-          tma_load_3d(sQ + st * C::kTileBytes + ch * C::kChunkBytes, &tm_q, &q_full[st], ch * 64,
-                      i * kBM, bh);
-        float *vec = sVec + st * C::kVecFloats;
-        bulk_load_1d(vec, p.lse2 + vec_row + i * kBM, kBM * 4, &q_full[st]);
-        bulk_load_1d(vec + kBM, p.dvec + vec_row + i * kBM, kBM * 4, &q_full[st]);
-        ++q_loads;
-        const int sd = t % C::kDoStages;
-        if (!mbar_wait(&do_empty[sd], ((t / C::kDoStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&do_full[sd], C::kTileBytes);
-        for (int ch = 0; ch < C::kChunks; ++ch)
-          tma_load_3d(sDO + sd * C::kTileBytes + ch * C::kChunkBytes, &tm_do, &do_full[sd],
-                      ch * 64, i * kBM, bh);
-        ++do_loads;
+      int q_loads = 0, do_loads = 0, kv_loads = 0;  // loads issued so far (= their global index)
+      for (int k = 0; ok; ++k) {
+        int bh, jb;
+        const int su = sub_unit(k, bh, jb);
+        if (su == 0) break;
+        if (su < 0) continue;
+        const Span sp = span_of(jb);
+        // K_j, V_j once every product of the previous sub-unit that read its K and V has completed.
+        // After the first sub-unit the query block t = 0 goes first: its Q and dO stages free up
+        // before the previous sub-unit's last dQ product releases K and V.
+        auto load_kv = [&]() -> bool {
+          if (kv_loads > 0 && !mbar_wait(kv_empty, (kv_loads - 1) & 1, abort_flag)) return false;
+          mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+          for (int ch = 0; ch < C::kChunks; ++ch) {
+            tma_load_3d(sK + ch * C::kChunkBytes, &tm_k, kv_full, ch * 64, jb * kBN, bh);
+            tma_load_3d(sV + ch * C::kChunkBytes, &tm_v, kv_full, ch * 64, jb * kBN, bh);
+          }
+          ++kv_loads;
+          return true;
+        };
+        bool kv_issued = false;
+        if (kv_loads == 0) {
+          if (!load_kv()) { ok = false; break; }
+          kv_issued = true;
+        }
+        const size_t vec_row = static_cast<size_t>(bh) * p.Np;
+        for (int t = 0; t < sp.n; ++t) {
+          const int i = sp.i_lo + (t + sp.rot) % sp.n;
+          const int g = q_loads, st = g % C::kStages;
+          const uint32_t ph = (g / C::kStages) & 1;
+          if (!mbar_wait(&q_empty[st], ph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[st], C::kTileBytes + C::kVecFloats * 4);
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            tma_load_3d(sQ + st * C::kTileBytes + ch * C::kChunkBytes, &tm_q, &q_full[st], ch * 64,
+                        i * kBM, bh);
+          float *vec = sVec + st * C::kVecFloats;
+          bulk_load_1d(vec, p.lse2 + vec_row + i * kBM, kBM * 4, &q_full[st]);
+          bulk_load_1d(vec + kBM, p.dvec + vec_row + i * kBM, kBM * 4, &q_full[st]);
+          ++q_loads;
+          const int sd = g % C::kDoStages;
+          if (!mbar_wait(&do_empty[sd], ((g / C::kDoStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&do_full[sd], C::kTileBytes);
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            tma_load_3d(sDO + sd * C::kTileBytes + ch * C::kChunkBytes, &tm_do, &do_full[sd],
+                        ch * 64, i * kBM, bh);
+          ++do_loads;
+          if (!kv_issued) {
+            if (!load_kv()) { ok = false; break; }
+            kv_issued = true;
+          }
+        }
       }
       if (!ok) {
         // abandoned: every copy already issued lands before the CTA's shared memory goes away
+        // (a K/V load is issued only after the previous one was consumed, so the last alone can
+        // be in flight)
         volatile int never = 0;
-        mbar_wait(kv_full, 0, &never);
+        if (kv_loads > 0) mbar_wait(kv_full, (kv_loads - 1) & 1, &never);
         for (int t = q_loads - C::kStages; t < q_loads; ++t)
           if (t >= 0) mbar_wait(&q_full[t % C::kStages], (t / C::kStages) & 1, &never);
         for (int t = do_loads - C::kDoStages; t < do_loads; ++t)
@@ -389,49 +418,66 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       const uint32_t sK0 = smem_u32(sK), sV0 = smem_u32(sV), sQ0 = smem_u32(sQ);
       const uint32_t sDO0 = smem_u32(sDO), sX0 = smem_u32(sX);
-      auto issue_s = [&](int t) -> bool {  // S^T_t = K_j Q_t^T into S^T's columns
-        const int st = t % C::kStages;
-        if (!mbar_wait(&q_full[st], (t / C::kStages) & 1, abort_flag)) return false;
-        if (t > 0 && !mbar_wait(s_free, (t - 1) & 1, abort_flag)) return false;
-        // d = 128: the columns held dQ_t-2 after S^T_t-1; it must have been read out
-        if (C::kDqT && t > 1 && !mbar_wait(dq_free, (t - 2) & 1, abort_flag)) return false;
+      // S^T_g = K_j Q_g^T into S^T's columns.  At d = 128 those columns also take the dQ^T
+      // partials.  Within a sub-unit S^T_g is issued before dQ^T_g-1 (which waits for S^T_g to be
+      // copied out), so S^T_g waits for dQ^T_g-2 to be read out; the first block of a sub-unit
+      // comes after the previous sub-unit's last dQ^T, g - 1, and waits for that one.
+      auto issue_s = [&](int g, bool first) -> bool {
+        const int st = g % C::kStages;
+        if (!mbar_wait(&q_full[st], (g / C::kStages) & 1, abort_flag)) return false;
+        if (g > 0 && !mbar_wait(s_free, (g - 1) & 1, abort_flag)) return false;
+        const int dq_prev = first ? g - 1 : g - 2;
+        if (C::kDqT && dq_prev >= 0 && !mbar_wait(dq_free, dq_prev & 1, abort_flag)) return false;
         tc_fence_after();
         issue_qk<HD>(tmem + C::kColS, sK0, sQ0 + st * C::kTileBytes);
         umma_commit(s_full);
         return true;
       };
-      auto issue_dp = [&](int t) -> bool {  // dP^T_t = V_j dO_t^T (dS^T_t-1 already formed)
-        const int sd = t % C::kDoStages;
-        if (!mbar_wait(&do_full[sd], (t / C::kDoStages) & 1, abort_flag)) return false;
+      auto issue_dp = [&](int g) -> bool {  // dP^T_g = V_j dO_g^T (dS^T_g-1 already formed)
+        const int sd = g % C::kDoStages;
+        if (!mbar_wait(&do_full[sd], (g / C::kDoStages) & 1, abort_flag)) return false;
         tc_fence_after();
         issue_qk<HD>(tmem + C::kColDP, sV0, sDO0 + sd * C::kTileBytes);
         umma_commit(dp_full);
         return true;
       };
-      bool ok = mbar_wait(kv_full, 0, abort_flag) && issue_s(0) && issue_dp(0);
-      for (int t = 0; ok && t < n; ++t) {
-        const int st = t % C::kStages, sd = t % C::kDoStages;
-        if (!mbar_wait(p_full, t & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        issue_x_kmajor<HD>(tmem + C::kColDV, sX0, sDO0 + sd * C::kTileBytes, C::kIdescKV, t > 0);
-        umma_commit(dv_done);
-        umma_commit(&do_empty[sd]);
-        if (t + 1 < n && !issue_s(t + 1)) { ok = false; break; }
-        if (!mbar_wait(ds_full, t & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        issue_x_kmajor<HD>(tmem + C::kColDK, sX0, sQ0 + st * C::kTileBytes, C::kIdescKV, t > 0);
-        umma_commit(&q_empty[st]);
-        // dQ_t-1 must have been read out of the dQ columns
-        if (t > 0 && !mbar_wait(dq_free, (t - 1) & 1, abort_flag)) { ok = false; break; }
-        if constexpr (C::kDqT) {
-          // dQ^T_t goes where S^T_t+1 sits: wait until the compute warps have copied it out
-          const int last_s = t + 1 < n ? t + 1 : t;
-          if (!mbar_wait(s_free, last_s & 1, abort_flag)) { ok = false; break; }
+      bool ok = true;
+      int T = 0, kv_used = 0;
+      for (int k = 0; ok; ++k) {
+        int bh, jb;
+        const int su = sub_unit(k, bh, jb);
+        if (su == 0) break;
+        if (su < 0) continue;
+        const int n = span_of(jb).n;
+        ok = mbar_wait(kv_full, kv_used & 1, abort_flag) && issue_s(T, true) && issue_dp(T);
+        ++kv_used;
+        for (int t = 0; ok && t < n; ++t) {
+          const int g = T + t, st = g % C::kStages, sd = g % C::kDoStages;
+          if (!mbar_wait(p_full, g & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_x_kmajor<HD>(tmem + C::kColDV, sX0, sDO0 + sd * C::kTileBytes, C::kIdescKV, t > 0);
+          umma_commit(dv_done);
+          umma_commit(&do_empty[sd]);
+          if (t + 1 < n && !issue_s(g + 1, false)) { ok = false; break; }
+          if (!mbar_wait(ds_full, g & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_x_kmajor<HD>(tmem + C::kColDK, sX0, sQ0 + st * C::kTileBytes, C::kIdescKV, t > 0);
+          umma_commit(&q_empty[st]);
+          // dQ_g-1 must have been read out of the dQ columns
+          if (g > 0 && !mbar_wait(dq_free, (g - 1) & 1, abort_flag)) { ok = false; break; }
+          if constexpr (C::kDqT) {
+            // dQ^T_g goes where S^T_g+1 sits: wait until the compute warps have copied it out
+            const int last_s = t + 1 < n ? g + 1 : g;
+            if (!mbar_wait(s_free, last_s & 1, abort_flag)) { ok = false; break; }
+          }
+          tc_fence_after();
+          issue_dq<HD>(tmem + C::kColDQ, sX0, sK0);
+          umma_commit(dq_full);
+          if (t + 1 < n && !issue_dp(g + 1)) { ok = false; break; }
         }
-        tc_fence_after();
-        issue_dq<HD>(tmem + C::kColDQ, sX0, sK0);
-        umma_commit(dq_full);
-        if (t + 1 < n && !issue_dp(t + 1)) { ok = false; break; }
+        if (!ok) break;
+        umma_commit(kv_empty);  // K_j and V_j are free once every product of the sub-unit has completed
+        T += n;
       }
       // every MMA issued by this thread completes before TMEM is released
       umma_commit(drain);
@@ -443,12 +489,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int w4 = warp % 4;
     const uint32_t tQ = tmem + (static_cast<uint32_t>(w4 * 32) << 16) + C::kColDQ;
     uint8_t *slot = sStage + w4 * C::kStageSlotBytes;
-    const int row_head = bh * p.Np;  // the head's first row in the accumulator's [BH * Np, d] view
-    for (int t = 0; t < n; ++t) {
-      const int i = qblock(t);
-      if (!__all_sync(0xffffffffu, mbar_wait(dq_full, t & 1, abort_flag))) break;
-      tc_fence_after();
-      read_out_dq<HD>(tQ, w4, lane, slot, &tm_dq, row_head + i * kBM, dq_free);
+    bool ok = true;
+    int T = 0;
+    for (int k = 0; ok; ++k) {
+      int bh, jb;
+      const int su = sub_unit(k, bh, jb);
+      if (su == 0) break;
+      if (su < 0) continue;
+      const Span sp = span_of(jb);
+      const int row_head = bh * p.Np;  // the head's first row in the accumulator's [BH * Np, d] view
+      for (int t = 0; t < sp.n; ++t) {
+        const int i = sp.i_lo + (t + sp.rot) % sp.n;
+        if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (T + t) & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+        read_out_dq<HD>(tQ, w4, lane, slot, &tm_dq, row_head + i * kBM, dq_free);
+      }
+      T += sp.n;
     }
     if (lane == 0) bulk_wait_group_all();  // every reduction has landed before the CTA retires
     __syncwarp();
@@ -461,119 +517,117 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tS = tmem + lane_off + C::kColS + 64 * h;
     const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * h;
     const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
-    const bool key_live = jb * kBN + r < p.N;  // keys past N (zero-filled rows) get P = 0
-    const bool ragged_keys = (jb + 1) * kBN > p.N;
     bool ok = true;
-    for (int t = 0; t < n; ++t) {
-      const int i = qblock(t), st = t % C::kStages;
-      const float *vlse = sVec + st * C::kVecFloats + 64 * h, *vd = vlse + kBM;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full, t & 1, abort_flag))) { ok = false; break; }
-      // S^T_t was computed from this stage, so it has landed; waiting makes its LSE2 / D rows
-      // visible to these threads
-      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], (t / C::kStages) & 1, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[64];
-      tmem_ld32(tS, reinterpret_cast<uint32_t *>(s));
-      tmem_ld32(tS + 32, reinterpret_cast<uint32_t *>(s) + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      // P^T: p = 2^(s scale log2(e) - LSE2_q); on the diagonal block (causal) key r is visible to
-      // query q only if r <= q, and keys past N are dropped
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 64; c += 4) {
-        const float4 l4 = *reinterpret_cast<const float4 *>(vlse + c);
-        const uint64_t x01 = f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, f2_pack(-l4.x, -l4.y));
-        const uint64_t x23 = f2_fma(f2_pack(s[c + 2], s[c + 3]), sl2x2, f2_pack(-l4.z, -l4.w));
-        float x0, x1, x2, x3;
-        f2_unpack(x01, x0, x1);
-        f2_unpack(x23, x2, x3);
-        s[c] = ex2(x0);
-        s[c + 1] = ex2(x1);
-        s[c + 2] = ex2(x2);
-        s[c + 3] = ex2(x3);
-      }
-      if ((p.causal && i == jb) || ragged_keys) {
-        const int qmin = r - 64 * h;  // visible iff local column >= qmin (diagonal block)
-        const bool diag = p.causal && i == jb;
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (!key_live || (diag && c < qmin)) s[c] = 0.f;
-      }
-#pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
-      if (t > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (t - 1) & 1, abort_flag))) { ok = false; break; }
-        tc_fence_after();
-      }
-      store_x_half(sX, r, h, pk);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-      // dS^T: ds = p (dP - D_q), with the bf16 p the tensor core used for dV
-      if (!__all_sync(0xffffffffu, mbar_wait(dp_full, t & 1, abort_flag))) { ok = false; break; }
-      tc_fence_after();
-      uint32_t dk[32];
-#pragma unroll
-      for (int cc = 0; cc < 64; cc += 32) {
-        uint32_t dp[32];
-        tmem_ld32(tDP + cc, dp);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 d4 = *reinterpret_cast<const float4 *>(vd + cc + e);
-          const uint32_t pa = pk[(cc + e) / 2], pb = pk[(cc + e) / 2 + 1];
-          const uint64_t g01 = f2_mul(f2_pack(__uint_as_float(pa << 16), __uint_as_float(pa & 0xffff0000u)),
-                                      f2_sub(f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
-                                             f2_pack(d4.x, d4.y)));
-          const uint64_t g23 = f2_mul(f2_pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xffff0000u)),
-                                      f2_sub(f2_pack(__uint_as_float(dp[e + 2]), __uint_as_float(dp[e + 3])),
-                                             f2_pack(d4.z, d4.w)));
-          float a0, a1, a2, a3;
-          f2_unpack(g01, a0, a1);
-          f2_unpack(g23, a2, a3);
-          dk[(cc + e) / 2] = pack_bf16x2(a0, a1);
-          dk[(cc + e) / 2 + 1] = pack_bf16x2(a2, a3);
+    int T = 0;
+    for (int k = 0; ok; ++k) {
+      int bh, jb;
+      const int su = sub_unit(k, bh, jb);
+      if (su == 0) break;
+      if (su < 0) continue;
+      const Span sp = span_of(jb);
+      const int n = sp.n;
+      const bool key_live = jb * kBN + r < p.N;  // keys past N (zero-filled rows) get P = 0
+      const bool ragged_keys = (jb + 1) * kBN > p.N;
+      for (int t = 0; t < n; ++t) {
+        const int g = T + t;
+        const int i = sp.i_lo + (t + sp.rot) % n, st = g % C::kStages;
+        const float *vlse = sVec + st * C::kVecFloats + 64 * h, *vd = vlse + kBM;
+        if (!__all_sync(0xffffffffu, mbar_wait(s_full, g & 1, abort_flag))) { ok = false; break; }
+        // S^T_g was computed from this stage, so it has landed; waiting makes its LSE2 / D rows
+        // visible to these threads
+        if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], (g / C::kStages) & 1, abort_flag))) {
+          ok = false;
+          break;
         }
-      }
-      tc_fence_before();
-      if (!__all_sync(0xffffffffu, mbar_wait(dv_done, t & 1, abort_flag))) { ok = false; break; }
-      store_x_half(sX, r, h, dk);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
-    }
-    // dV_j and dK_j (times scale) once every MMA has completed
-    if (ok && __all_sync(0xffffffffu, mbar_wait(dq_full, (n - 1) & 1, abort_flag))) {
-      tc_fence_after();
-      if (HD == 128 && p.g_tma) {
-        // each warp's 32 key rows x 64 features of dV and dK: staged in the Q ring (every MMA
-        // that read it has completed) and written with one tensor store each, clipped at row N
-        uint8_t *box_v = sQ + warp * 4096, *box_k = sQ + 8 * 4096 + warp * 4096;
-        stage_grad_box(tmem + lane_off + C::kColDV, h * 64, 1.f, box_v, lane);
-        stage_grad_box(tmem + lane_off + C::kColDK, h * 64, p.scale, box_k, lane);
+        tc_fence_after();
+        float s[64];
+        tmem_ld32(tS, reinterpret_cast<uint32_t *>(s));
+        tmem_ld32(tS + 32, reinterpret_cast<uint32_t *>(s) + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        // P^T: p = 2^(s scale log2(e) - LSE2_q); on the diagonal block (causal) key r is visible
+        // to query q only if r <= q, and keys past N are dropped
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4 *>(vlse + c);
+          const uint64_t x01 = f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, f2_pack(-l4.x, -l4.y));
+          const uint64_t x23 = f2_fma(f2_pack(s[c + 2], s[c + 3]), sl2x2, f2_pack(-l4.z, -l4.w));
+          float x0, x1, x2, x3;
+          f2_unpack(x01, x0, x1);
+          f2_unpack(x23, x2, x3);
+          s[c] = ex2(x0);
+          s[c + 1] = ex2(x1);
+          s[c + 2] = ex2(x2);
+          s[c + 3] = ex2(x3);
+        }
+        if ((p.causal && i == jb) || ragged_keys) {
+          const int qmin = r - 64 * h;  // visible iff local column >= qmin (diagonal block)
+          const bool diag = p.causal && i == jb;
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (!key_live || (diag && c < qmin)) s[c] = 0.f;
+        }
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
+        // X still feeds the previous block's dQ product (the previous sub-unit's last one was
+        // waited for before its gradients were written)
+        if (t > 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (g - 1) & 1, abort_flag))) { ok = false; break; }
+          tc_fence_after();
+        }
+        store_x_half(sX, r, h, pk);
         fence_async_smem();
         __syncwarp();
-        const int r0 = jb * kBN + 32 * w4;
-        if (lane == 0 && r0 < p.N) {
-          tma_store_3d(&tm_dv, box_v, 64 * h, r0, bh);
-          tma_store_3d(&tm_dk, box_k, 64 * h, r0, bh);
-          bulk_commit_group();
-          bulk_wait_group_all();  // the boxes have been read before the CTA retires
+        if (lane == 0) mbar_arrive(p_full);
+        // dS^T: ds = p (dP - D_q), with the bf16 p the tensor core used for dV
+        if (!__all_sync(0xffffffffu, mbar_wait(dp_full, g & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t dk[32];
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 32) {
+          uint32_t dp[32];
+          tmem_ld32(tDP + cc, dp);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 d4 = *reinterpret_cast<const float4 *>(vd + cc + e);
+            const uint32_t pa = pk[(cc + e) / 2], pb = pk[(cc + e) / 2 + 1];
+            const uint64_t g01 = f2_mul(f2_pack(__uint_as_float(pa << 16), __uint_as_float(pa & 0xffff0000u)),
+                                        f2_sub(f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                               f2_pack(d4.x, d4.y)));
+            const uint64_t g23 = f2_mul(f2_pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xffff0000u)),
+                                        f2_sub(f2_pack(__uint_as_float(dp[e + 2]), __uint_as_float(dp[e + 3])),
+                                               f2_pack(d4.z, d4.w)));
+            float a0, a1, a2, a3;
+            f2_unpack(g01, a0, a1);
+            f2_unpack(g23, a2, a3);
+            dk[(cc + e) / 2] = pack_bf16x2(a0, a1);
+            dk[(cc + e) / 2 + 1] = pack_bf16x2(a2, a3);
+          }
         }
+        tc_fence_before();
+        if (!__all_sync(0xffffffffu, mbar_wait(dv_done, g & 1, abort_flag))) { ok = false; break; }
+        store_x_half(sX, r, h, dk);
+        fence_async_smem();
         __syncwarp();
-      } else {
-        const size_t grow = static_cast<size_t>(bh) * p.N + jb * kBN + r;
-        store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDV, h * (HD / 2), 1.f, p.dv,
-                                     p.g_f32, grow, key_live);
-        store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDK, h * (HD / 2), p.scale, p.dk,
-                                     p.g_f32, grow, key_live);
+        if (lane == 0) mbar_arrive(ds_full);
       }
+      if (!ok) break;
+      // dV_j and dK_j (times scale) once every product of the sub-unit has completed.  The next
+      // sub-unit's first dV and dK products overwrite these columns; the issuer starts them only
+      // after this warp's next P^T / dS^T signals, i.e. after these reads.
+      if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (T + n - 1) & 1, abort_flag))) { ok = false; break; }
+      tc_fence_after();
+      const size_t grow = static_cast<size_t>(bh) * p.N + jb * kBN + r;
+      store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDV, h * (HD / 2), 1.f, p.dv, p.g_f32,
+                                   grow, key_live);
+      store_grad_cols<HD, HD / 64>(tmem + lane_off + C::kColDK, h * (HD / 2), p.scale, p.dk,
+                                   p.g_f32, grow, key_live);
+      tc_fence_before();
+      T += n;
     }
   }
 

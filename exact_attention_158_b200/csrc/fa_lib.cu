@@ -341,14 +341,10 @@ fa_status launch_bwd(DeviceInfo &dev, const void *q, const void *k, const void *
     t_last_error = "cuTensorMapEncodeTiled failed";
     return FA_ERR_LAUNCH;
   }
-  // d = 128, bf16 dK / dV: tensor stores of 32-row boxes (without the maps the kernel never reads
-  // its dK / dV map arguments)
-  CUtensorMap tdk, tdv;
-  p.g_tma = (HD == 128 && !g_f32 && encode_bhnd(&tdk, dk, HD, N, BH, 32) &&
-             encode_bhnd(&tdv, dv, HD, N, BH, 32)) ? 1 : 0;
-  const long long units = static_cast<long long>(BH) * p.nkb;
-  fa::fa_bwd_kernel<HD><<<static_cast<unsigned>(units), fa::kBwdThreads, C::kSmemBytes, stream>>>(
-      tq, tk, tv, tdo, tdq, p.g_tma ? tdk : tq, p.g_tma ? tdv : tq, p);
+  // persistent: one CTA per SM at most, each taking pairs of key blocks (see the kernel)
+  const long long pairs = static_cast<long long>(BH) * ((p.nkb + 1) / 2);
+  const unsigned grid = static_cast<unsigned>(pairs < dev.num_sms ? pairs : dev.num_sms);
+  fa::fa_bwd_kernel<HD><<<grid, fa::kBwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return launch_failed(e);
   const long long post_threads = static_cast<long long>(BH) * N * kRowThreads;
   fa::fa_bwd_dq_kernel<HD><<<static_cast<unsigned>((post_threads + 255) / 256), 256, 0, stream>>>(
