@@ -11,22 +11,22 @@
 //
 // B200 mapping (one CTA per SM, 384 threads, persistent over work units):
 //   warps 0-3   softmax for query tile 0 of the current pair (one TMEM lane = one query row)
-//   warps 4-7   softmax for query tile 1 of the pair
+//   warps 4-7   softmax for query tile 1 of the pair; warp w and warp w + 4 share an SM
+//               sub-partition and take turns on its exponential unit
 //   warp  8     TMA producer: the Q pair once per unit, then K_0, and K_{j+1}, V_j per block
-//   warp  9     MMA issuer (one thread) + TMEM owner
-//   warps 10-11 idle
-// TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+d)  O1 [256+d, 256+2d), and at d = 64
-// also P0, P1 (64 columns each: two bf16 per column).
-// P_i (bf16) is written by the softmax threads into its own buffer (TMEM at d = 64, shared memory
-// in the layout the tensor core reads at d = 128), so S_i's TMEM columns are free as soon as the
-// softmax has copied S_i,j into registers:
-// the MMA warp then computes S_i,j+1 while the softmax is still turning S_i,j into P_i,j, and
-// O_i += P_i,j V_j follows when P_i,j is ready.  Each softmax warpgroup thus runs back to back,
-// and the two tiles keep the tensor core fed in turn.
+//   warp  9     Q K^T issuer (one thread) + TMEM owner
+//   warp  10    P V issuer (one thread); in the paged mode it first ranks the sequences
+//   warp  11    idle
+// TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+d)  O1 [256+d, 256+2d).
+// P_i (bf16) is written by the softmax threads into a shared-memory tile in the layout the tensor
+// core reads, so S_i's TMEM columns are free as soon as the softmax has copied S_i,j into
+// registers: the Q K^T issuer then computes S_i,j+1 while the softmax is still turning S_i,j into
+// P_i,j, and the P V issuer adds O_i += P_i,j V_j when P_i,j is ready.  Each softmax warpgroup
+// thus runs back to back, and the two tiles keep the tensor core fed in turn.
 // Epilogue: O_i / l_i per row.  In the square and paged modes with bf16 O each warp stages its
-// 32 rows in shared memory (d = 128: the then unused P buffer; d = 64: a staging tile of its own)
-// and writes them with TMA tensor stores, so the warp starts the next unit while the stores drain;
-// otherwise every thread stores its own row.
+// 32 rows in the tile's P buffer (free once the last P V has completed) and writes them with TMA
+// tensor stores, so the warp starts the next unit while the stores drain; otherwise every thread
+// stores its own row.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -80,8 +80,8 @@ struct PrefillCfg {
   // unit busy without contention.
   static constexpr bool kExpTurns = FA_EXP_TURNS != 0;
   static constexpr int kPBytes = kPInTmem ? 0 : 128 * kBN * 2;  // one 128 x 128 bf16 P tile
-  // bf16 O staging for the tensor-store epilogue: the P tile where there is one, else a buffer of
-  // its own per query tile (d = 64: 128 rows x 128 bytes)
+  // bf16 O staging for the tensor-store epilogue: the P tile where there is one (both head dims
+  // as built), else a buffer of its own per query tile (128 rows x d bf16)
   static constexpr int kOStageBytes = kPInTmem ? 128 * HD * 2 : 0;
   // K/V ring depth: K_{j+1} is loaded one block ahead of V_j, so three stages give every load
   // about one block of slack.
@@ -767,9 +767,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                    : static_cast<size_t>(w.bh) * p.N + qrow;
       if (kTmaO && p.o_tma) {
         // O / l as bf16 into this thread's row of the staging tile (the layout P uses: 64 columns
-        // per 128-byte-swizzled chunk), then one tensor store per chunk of the warp's 32 rows.  A
-        // staging tile of its own (d = 64) still holds this warp's rows of the previous unit's O
-        // until those stores have read it.
+        // per 128-byte-swizzled chunk), then one tensor store per chunk of the warp's 32 rows.  With
+        // P in TMEM (kPInTmem, not the configuration built) the staging tile is a buffer of its
+        // own that still holds this warp's rows of the previous unit's O until those stores have
+        // read it.
         if constexpr (C::kPInTmem) {
           if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
