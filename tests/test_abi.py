@@ -98,6 +98,8 @@ def test_prefill_paged_rejections(lib):
     assert pp(lib, q=A + 8) == 3 and pp(lib, table=5 * A + 2) == 3 and pp(lib, lens=6 * A + 1) == 3
     assert pp(lib, o=A + 32) == 1  # output overlaps q
     assert pp(lib, o=2 * A + 64) == 1  # output overlaps the K pool
+    # (block, head) pages are indexed as block * H + head in an int: (num_blocks + 1) * H must fit
+    assert pp(lib, P=2 ** 30, H=2) == 1
 
 
 def bwd(lib, dq=8 * A, ws=12 * A, ws_bytes=1 << 30, B=1, H=2, N=300, d=128, causal=0, dt=0,
