@@ -22,6 +22,17 @@ def test_backward_multi_tile(causal):
     parity.run_backward(W.PrefillCase("bwd_multi", 2, 3, 1024, 128, causal))
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_persistent_odd_key_blocks(causal, d):
+    # N = 300: three key blocks per head (the middle pair is a single sub-unit, the last block is
+    # ragged); 160 heads make 320 pairs, so each of the persistent CTAs walks two or three pairs
+    # and carries its barrier phases across sub-units of different lengths.  Heads spread over
+    # the CTAs are checked in full.
+    parity.run_backward(W.PrefillCase(f"bwd_pers_d{d}", 4, 40, 300, d, causal),
+                        heads=[0, 1, 73, 148, 149, 159])
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_backward_config_sampled_heads(causal):
     # the bench's training-shape configuration (B8 H16 N2048 d128), three heads checked in full
@@ -36,7 +47,7 @@ def test_backward_bf16_grads(d):
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 33, 129, 257, 1000])
 def test_backward_ragged_bf16_grads(N, causal):
-    # bf16 dK / dV at d = 128 leave through tensor stores of 32-row boxes, clipped at row N
+    # bf16 dK / dV, rows past N never written
     parity.run_backward(W.PrefillCase(f"bwd_bf16_N{N}", 1, 3, N, 128, causal),
                         grad_dtype=torch.bfloat16)
 
