@@ -111,15 +111,21 @@ def test_pool_relocation_is_bitwise_invariant():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def test_bad_block_id_is_reported_not_read():
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bad", ["past_pool", "negative"])
+def test_bad_block_id_is_reported_not_read(d, bad):
+    # d = 128 gathers whole pages through a map indexed block * H + head: an entry past the pool
+    # or negative must still land out of range (zeros), never on another head's or block's page
     import exact_attention_158_b200 as fa
-    case = W.DecodeCase("pp_bad", S=2, H=2, d=64, lens=[200, 64])
+    case = W.DecodeCase("pp_bad", S=2, H=2, d=d, lens=[200, 64])
     inp = W.make_paged_prefill(case, 16, device="cuda")
     table = inp["block_table"].clone()
-    table[0, 3] = inp["num_blocks"] + 1000
-    fa.fa_prefill_paged(inp["q"], inp["k_pool"], inp["v_pool"], table, inp["seq_lens"])
+    table[0, 3] = inp["num_blocks"] + 1000 if bad == "past_pool" else -7
+    o, lse = fa.fa_prefill_paged(inp["q"], inp["k_pool"], inp["v_pool"], table, inp["seq_lens"],
+                                 out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert fa.device_status() == 1  # FA_ERR_INVALID_ARG
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
     # the error word is cleared by the read; a good call afterwards reports nothing
     fa.fa_prefill_paged(inp["q"], inp["k_pool"], inp["v_pool"], inp["block_table"],
                         inp["seq_lens"])
