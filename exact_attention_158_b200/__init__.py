@@ -34,7 +34,7 @@ EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode_workspace_size", "fa_decode_paged",
                     "fa_bwd", "fa_get_device_status",
                     "fa_status_string",
                     "fa_last_error_string", "fa_version", "fa_selftest_wait_timeout",
-                    "fa_probe_ex2_rate", "fa_probe_read_rate")
+                    "fa_probe_ex2_rate", "fa_probe_read_rate", "fa_fwd_schedule")
 
 _lib = None
 
@@ -456,3 +456,22 @@ def probe_read_rate(buf: torch.Tensor, stream=None) -> float:
     b.record(s)
     b.synchronize()
     return a.elapsed_time(b)
+
+
+def fwd_schedule(B: int, H: int, N: int, d: int, num_ctas: int):
+    """The unit-to-CTA assignment of a causal fa_fwd launch of this shape on `num_ctas` SMs (host
+    only).  Returns (start, unit) int32 numpy arrays, CTA c running unit[start[c]:start[c+1]] in
+    order, or None when the launch deals its units in snake order instead."""
+    import numpy as np
+    lib = load_library()
+    f = lib.fa_fwd_schedule
+    ip = ctypes.POINTER(ctypes.c_int)
+    f.argtypes = [ctypes.c_int] * 5 + [ip, ip, ctypes.c_int, ip]
+    f.restype = ctypes.c_int
+    units = B * H * ((N + 255) // 256)
+    start = np.zeros(num_ctas + 1, dtype=np.int32)
+    unit = np.zeros(max(units, 1), dtype=np.int32)
+    count = ctypes.c_int(0)
+    _check(f(B, H, N, d, num_ctas, start.ctypes.data_as(ip), unit.ctypes.data_as(ip), unit.size,
+             ctypes.byref(count)), "fa_fwd_schedule")
+    return (start, unit[:count.value]) if count.value > 0 else None

@@ -12,6 +12,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "fa.h"
 #include "fa_backward.cuh"
@@ -226,6 +227,78 @@ bool encode_pool_v_pages(CUtensorMap *map, const void *base, int H, int num_bloc
   return r == CUDA_SUCCESS;
 }
 
+// Static unit assignment of a causal square launch (fa::UnitTable).  The units are taken in groups
+// of heads whose K and V total at most kGroupKvBytes (a quarter of L2), longest pair level first
+// within a group, and each goes to the CTA that frees up first under the cost model "key blocks of
+// both tiles + 1.5" (ties to the lowest CTA).  A group keeps at least kMinGroupHeads heads (with
+// fewer, dozens of CTAs stream the same head's K/V at once, which measured slower) and there are
+// no more groups than full rounds of units.  Returns false when the launch takes no table (d = 64,
+// see fa::UnitTableOf; or one group: the level-major snake is then as good).
+constexpr double kGroupKvBytes = 32.0 * 1024 * 1024;
+constexpr int kMinGroupHeads = 16;
+
+static bool build_unit_table(fa::UnitTable &t, int BH, int N, int num_pairs, int grid, int HD) {
+  const int units = BH * num_pairs;
+  if (HD != 128 || grid <= 0 || grid > fa::kMaxSchedCtas || units <= grid || units > fa::kMaxSchedUnits)
+    return false;
+  const double kv_head = 2.0 * N * HD * 2;  // bf16 K and V of one (b, h)
+  int groups = static_cast<int>(std::ceil(BH * kv_head / kGroupKvBytes));
+  groups = std::min({groups, units / grid, BH / kMinGroupHeads});
+  if (groups <= 1) return false;
+  auto tile_blocks = [&](int pr, int i) {
+    const int q0 = pr * 2 * fa::kBM + i * fa::kBM;
+    return q0 >= N ? 0 : (std::min(q0 + fa::kBM, N) - 1) / fa::kBN + 1;
+  };
+  std::vector<int> owner(units);
+  std::vector<int> order;
+  order.reserve(units);
+  std::vector<std::pair<long, int>> heap;  // (finish time in half blocks, CTA): a min-heap
+  for (int c = 0; c < grid; ++c) heap.push_back({0, c});
+  auto later = [](const std::pair<long, int> &a, const std::pair<long, int> &b) { return a > b; };
+  std::make_heap(heap.begin(), heap.end(), later);
+  for (int g = 0, h0 = 0; g < groups; ++g) {
+    const int gk = BH / groups + (g < BH % groups ? 1 : 0);
+    for (int level = 0; level < num_pairs; ++level) {
+      const int pr = num_pairs - 1 - level;
+      const long cost = 2L * (tile_blocks(pr, 0) + tile_blocks(pr, 1)) + 3;
+      for (int bh = h0; bh < h0 + gk; ++bh) {
+        std::pop_heap(heap.begin(), heap.end(), later);
+        const int u = level * BH + bh;
+        owner[u] = heap.back().second;
+        order.push_back(u);
+        heap.back().first += cost;
+        std::push_heap(heap.begin(), heap.end(), later);
+      }
+    }
+    h0 += gk;
+  }
+  std::vector<int> count(grid + 1, 0);
+  for (int u = 0; u < units; ++u) ++count[owner[u] + 1];
+  for (int c = 0; c < grid; ++c) count[c + 1] += count[c];
+  for (int c = 0; c <= grid; ++c) t.start[c] = static_cast<uint16_t>(count[c]);
+  std::vector<int> fill(count.begin(), count.end() - 1);
+  for (int u : order) t.unit[fill[owner[u]]++] = static_cast<uint16_t>(u);  // per CTA in run order
+  t.count = units;
+  return true;
+}
+
+// The table of the last causal square launch made by this thread, reused while the shape repeats.
+struct UnitTableCache {
+  int BH = -1, N = -1, grid = -1, HD = -1;
+  bool valid = false;
+  fa::UnitTable table{};
+};
+
+static const fa::UnitTable &unit_table(int BH, int N, int num_pairs, int grid, int HD) {
+  static thread_local UnitTableCache cache;
+  static const fa::UnitTable none{};
+  if (cache.BH != BH || cache.N != N || cache.grid != grid || cache.HD != HD) {
+    cache.BH = BH, cache.N = N, cache.grid = grid, cache.HD = HD;
+    cache.valid = build_unit_table(cache.table, BH, N, num_pairs, grid, HD);
+  }
+  return cache.valid ? cache.table : none;
+}
+
 template <int HD, int kMode>
 fa_status launch_prefill(DeviceInfo &dev, const CUtensorMap &tq, const CUtensorMap &tk,
                          const CUtensorMap &tv, fa::PrefillParams p, cudaStream_t stream,
@@ -246,8 +319,12 @@ fa_status launch_prefill(DeviceInfo &dev, const CUtensorMap &tq, const CUtensorM
   }
   const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
   // without an O map (p.o_tma = 0) the kernel never reads its O map argument
+  typename fa::UnitTableOf<HD, kMode>::type tab{};
+  if constexpr (!std::is_same_v<decltype(tab), fa::NoUnitTable>) {
+    if (p.causal) tab = unit_table(p.BH, p.N, p.num_pairs, grid, HD);
+  }
   fa::fa_prefill_kernel<HD, kMode><<<grid, fa::kPrefillThreads, C::kSmemBytes, stream>>>(
-      tq, tk, tv, to != nullptr ? *to : tq, p);
+      tq, tk, tv, to != nullptr ? *to : tq, p, tab);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : launch_failed(e);
 }
@@ -873,6 +950,26 @@ const char *fa_status_string(fa_status status) {
 }
 
 const char *fa_last_error_string(void) { return t_last_error.c_str(); }
+
+fa_status fa_fwd_schedule(int B, int H, int N, int d, int num_ctas, int *start, int *unit,
+                          int capacity, int *count) {
+  if (count == nullptr || start == nullptr || unit == nullptr) return FA_ERR_INVALID_ARG;
+  *count = 0;
+  if (B < 1 || H < 1 || N < 1 || num_ctas < 1 || num_ctas > 1024) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
+  const long long pairs = (static_cast<long long>(N) + 2 * fa::kBM - 1) / (2 * fa::kBM);
+  if (BH * pairs > INT_MAX) return FA_ERR_INVALID_ARG;
+  const int units = static_cast<int>(BH * pairs);
+  if (capacity < units) return FA_ERR_INVALID_ARG;
+  const int grid = std::min(units, num_ctas);
+  static thread_local fa::UnitTable t;
+  if (!build_unit_table(t, static_cast<int>(BH), N, static_cast<int>(pairs), grid, d)) return FA_OK;
+  for (int c = 0; c <= num_ctas; ++c) start[c] = c <= grid ? t.start[c] : units;
+  for (int i = 0; i < units; ++i) unit[i] = t.unit[i];
+  *count = units;
+  return FA_OK;
+}
 
 int fa_version(void) { return kVersion; }
 

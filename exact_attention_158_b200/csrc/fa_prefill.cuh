@@ -28,6 +28,8 @@
 // tensor stores, so the warp starts the next unit while the stores drain; otherwise every thread
 // stores its own row.
 #pragma once
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -158,6 +160,13 @@ __device__ __forceinline__ KvSpan kv_span(const PrefillParams &p, int bh) {
 // numbered from the most expensive pair level down (unit = level * BH + bh, pair = pairs-1-level)
 // and dealt to the CTAs in snake order (round r gives CTA c the unit r*G + c for even r and
 // r*G + G-1-c for odd r), a static form of longest-processing-time-first scheduling.
+//
+// That order keeps every head's K and V in play at once, more than L2 holds at N >= 2k, so causal
+// launches re-read K/V from DRAM.  At d = 128, up to kMaxSchedUnits units, the host instead passes
+// a UnitTable:
+// list scheduling (each unit to the CTA that frees up first, under the cost above) over the units
+// taken in groups of heads whose K and V fill a fraction of L2, longest first within a group.  It
+// balances the CTAs as well as the snake and keeps about one group of heads in flight.
 struct WorkUnit {
   int bh;
   int pair;
@@ -170,11 +179,35 @@ struct WorkUnit {
 // key-range mode, units are numbered head-major and dealt round-robin.
 constexpr int kMaxSortedSeqs = 128;
 
+constexpr int kMaxSchedUnits = 2048;
+constexpr int kMaxSchedCtas = 160;
+
+// Causal square launches: CTA c runs the units unit[start[c]] .. unit[start[c+1] - 1] in that
+// order (unit numbers as in the level-major numbering above).  count = 0: no table.
+struct UnitTable {
+  int count;
+  uint16_t start[kMaxSchedCtas + 1];
+  uint16_t unit[kMaxSchedUnits];
+};
+
+// Only the d = 128 square instance takes a table.  The paged and key-range modes order their units
+// otherwise; at d = 64 the kernel is bound by its exponentials, so DRAM re-reads cost it nothing,
+// while the table lookup made that instance spill (2-5% slower, non-causal launches included).
+struct NoUnitTable {};
+template <int HD, int kMode> struct UnitTableOf { using type = NoUnitTable; };
+template <> struct UnitTableOf<128, kModeSquare> { using type = UnitTable; };
+
 // The unit CTA blockIdx.x processes in its round r, or -1 once it has none left.
-template <bool kGeneral = false>
-__device__ __forceinline__ int unit_for_round(const PrefillParams &p, int r,
+template <bool kGeneral, class Table>
+__device__ __forceinline__ int unit_for_round(const PrefillParams &p, const Table &tab, int r,
                                               const int *seq_order = nullptr) {
   const int G = gridDim.x, c = blockIdx.x;
+  if constexpr (!std::is_same_v<Table, NoUnitTable>) {
+    if (tab.count > 0) {
+      const int i = tab.start[c] + r;
+      return i < tab.start[c + 1] ? tab.unit[i] : -1;
+    }
+  }
   const bool snake = kGeneral ? seq_order != nullptr : p.causal;
   const int u = r * G + ((snake && (r & 1)) ? G - 1 - c : c);
   return u < p.num_units ? u : -1;
@@ -320,7 +353,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
+                      const __grid_constant__ CUtensorMap tm_o, const PrefillParams p,
+                      const __grid_constant__ typename UnitTableOf<HD, kMode>::type tab) {
   using C = PrefillCfg<HD>;
   constexpr bool kPaged = kMode == kModePaged;
   constexpr bool kGeneral = kMode != kModeSquare;  // key count and query offset per unit
@@ -473,7 +507,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         return true;
       };
       for (int r = 0; ok; ++r) {
-        const int u = unit_for_round<kGeneral>(p, r, seq_order);
+        const int u = unit_for_round<kGeneral>(p, tab, r, seq_order);
         if (u < 0) break;
         const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
         const int pr = w.pair;
@@ -529,7 +563,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       };
       bool ok = true;
       for (int r = 0; ok; ++r) {
-        const int u = unit_for_round<kGeneral>(p, r, seq_order);
+        const int u = unit_for_round<kGeneral>(p, tab, r, seq_order);
         if (u < 0) break;
         const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
         const KvSpan kv = kv_span<kMode>(p, w.bh);
@@ -616,7 +650,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     };
     if (C::kExpTurns && wg == 1) pass_turn();
     for (int r = 0; ok; ++r) {
-      const int u = unit_for_round<kGeneral>(p, r, seq_order);
+      const int u = unit_for_round<kGeneral>(p, tab, r, seq_order);
       if (u < 0) break;
       const WorkUnit w = decode_unit<kGeneral>(p, u, seq_order);
       const int pr = w.pair;

@@ -314,6 +314,29 @@ fa_status fa_probe_ex2_rate(float *sink, int iters, long long *exps_out, fa_stre
  */
 fa_status fa_probe_read_rate(const void *buf, size_t bytes, float *sink, fa_stream_t stream);
 
+/*
+ * fa_fwd_schedule -- host only: the assignment of work units to CTAs that a causal fa_fwd launch
+ * of this shape makes on a GPU with num_ctas SMs; no device is touched.  Work is split over batch,
+ * head and query tile ("FlashAttention-2 GPU work partitioning", section 3): a unit is one pair of
+ * 128-row query tiles of one (b, h), numbered level-major, so unit u covers (b*H + h) = u % (B*H)
+ * and query tiles 2p and 2p + 1 with p = ceil(N / 256) - 1 - u / (B*H); its cost grows with p.
+ * At d = 128 the launch balances the CTAs by list scheduling over heads taken in groups whose K and
+ * V fill a fraction of L2, longest units first within a group, so that one group's K and V stay
+ * resident; at d = 64 (bound by its exponentials, not by DRAM) it always deals in snake order.
+ *
+ *   B, H, N, d  as for fa_fwd (d: 64 or 128);  num_ctas in 1 .. 1024.
+ *   start       int [num_ctas + 1], host memory: CTA c runs unit[start[c]] .. unit[start[c+1] - 1]
+ *               in that order.  Entries past the launch's CTA count G = min(units, num_ctas) are
+ *               set to the unit count.
+ *   unit        int [capacity], host memory.
+ *   *count      the number of units in the table, or 0 when the launch takes no table: it then
+ *               deals the units in snake order (round r gives CTA c unit r*G + c for even r and
+ *               r*G + G-1-c for odd r), and start / unit are not written.
+ * FA_ERR_INVALID_ARG for bad sizes, null pointers, or a capacity below the unit count.
+ */
+fa_status fa_fwd_schedule(int B, int H, int N, int d, int num_ctas, int *start, int *unit,
+                          int capacity, int *count);
+
 /* Static text for a status code. */
 const char *fa_status_string(fa_status status);
 

@@ -45,6 +45,28 @@ def test_prefill_config(causal, out_dtype):
     parity.run_prefill(W.PrefillCase("prefill", 8, 16, 2048, 128, causal), out_dtype)
 
 
+@pytest.mark.parametrize("shape", [(8, 16, 2048, 128), (32, 16, 512, 128), (4, 16, 4096, 128)],
+                         ids=lambda s: "B{}H{}N{}d{}".format(*s))
+def test_scheduled_causal_writes_every_row(shape):
+    # causal launches of these shapes run their units from a host-built table (fa_fwd_schedule):
+    # every row must be written (the outputs start as NaN), and row 0 of each head, which sees key
+    # 0 alone, is V's row 0 with LSE = scale * q_0 . k_0
+    import math
+    import exact_attention_158_b200 as fa
+    B, H, N, d = shape
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert fa.fwd_schedule(B, H, N, d, sms) is not None
+    q, k, v = W.make_prefill(W.PrefillCase("sched", B, H, N, d, True), device="cuda")
+    o = torch.full((B, H, N, d), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device="cuda")
+    fa.fa_fwd(q, k, v, causal=True, out_dtype=torch.float32, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all(), "a unit was never run"
+    torch.testing.assert_close(o[:, :, 0, :], v[:, :, 0, :].float(), rtol=1e-6, atol=1e-6)
+    s00 = (q[:, :, 0, :].double() * k[:, :, 0, :].double()).sum(-1) / math.sqrt(d)
+    torch.testing.assert_close(lse[:, :, 0].double(), s00, rtol=1e-5, atol=1e-5)
+
+
 @pytest.mark.parametrize("case", W.sweep_cases(128) + W.sweep_cases(64),
                          ids=lambda c: f"{c.name}_N{c.N}_{'causal' if c.causal else 'full'}")
 def test_sweep(case):
