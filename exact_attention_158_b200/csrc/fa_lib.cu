@@ -175,7 +175,8 @@ bool resolve_scale(float scale, int d, float *out) {
 }
 
 // The pools [num_blocks, H, 16, d] as a 4-D tensor (d, 16, H, num_blocks) read in 64 x 16 x 1 x 1
-// boxes: one 16-token page of one head per load.
+// boxes.  Used at d = 64, where that box is a whole 16-token page of one head (2 KB); d = 128 takes
+// the 5-D page maps below.
 bool encode_pool(CUtensorMap *map, const void *base, int d, int H, int num_blocks) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;

@@ -346,8 +346,10 @@ __device__ __forceinline__ void store_p_row(uint8_t *p_tile, int row, const uint
   }
 }
 
-// kMode: kModeSquare, kModePaged (tm_k / tm_v are 4-D maps over the pools [num_blocks, H, 16, d];
-// a 128-key tile is gathered as eight 16-row pages through the block table) or kModeRange.
+// kMode: kModeSquare, kModePaged (tm_k / tm_v map the pools [num_blocks, H, 16, d]; a 128-key
+// tile is gathered as eight 16-row pages through the block table, one TMA box per page: 4-D maps
+// at d = 64, 5-D maps at d = 128 whose box reorders the page into the operand layout) or
+// kModeRange.
 template <int HD, int kMode>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
