@@ -63,7 +63,9 @@ def mean_live_heads(lists, BH, N, samples=400):
 
 # (B, H, N, d): the causal shapes of the forward's benchmark and its sequence-length sweep
 TABLE_SHAPES = [(8, 16, 2048, 128), (4, 16, 4096, 128), (32, 16, 512, 128), (16, 16, 1024, 128),
-                (2, 16, 8192, 128), (1, 32, 16384, 128)]
+                (2, 16, 8192, 128), (1, 32, 16384, 128),
+                # ragged N: the last pair's second tile is short or empty
+                (8, 16, 1900, 128), (3, 32, 4000, 128), (6, 16, 3000, 128)]
 
 
 @pytest.mark.parametrize("shape", TABLE_SHAPES, ids=lambda s: "B{}H{}N{}d{}".format(*s))
