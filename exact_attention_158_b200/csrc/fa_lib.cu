@@ -448,6 +448,10 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, fa_out_dt
   if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  // work units (pairs of 128-row query tiles) are counted in an int
+  if (static_cast<long long>(B) * H * ((static_cast<long long>(N) + 2 * fa::kBM - 1) / (2 * fa::kBM)) >
+      INT_MAX)
+    return FA_ERR_INVALID_ARG;
   float sc;
   if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;
@@ -798,6 +802,10 @@ fa_status fa_fwd_keyrange(const void *q, const void *k, const void *v, void *o, 
   if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_F32) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  // work units (pairs of 128-row query tiles) are counted in an int
+  if (static_cast<long long>(B) * H * ((static_cast<long long>(Nq) + 2 * fa::kBM - 1) / (2 * fa::kBM)) >
+      INT_MAX)
+    return FA_ERR_INVALID_ARG;
   float sc;
   if (!resolve_scale(scale, d, &sc)) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;

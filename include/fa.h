@@ -65,7 +65,7 @@ typedef enum {
  *   o         [B, H, N, d] contiguous, bf16 or fp32 per o_dtype.  16-byte aligned.  Must not
  *             overlap q, k, v or lse.
  *   lse       fp32 [B, H, N] (natural log of the row sum of exp(scaled scores)), or NULL.
- *   B, H, N   >= 1;  B*H*N*d must fit in int64;  B*H < 2^31;  N < 2^31.
+ *   B, H, N   >= 1;  B*H*N*d must fit in int64;  B*H < 2^31;  B*H*ceil(N/256) < 2^31;  N < 2^31.
  *   d         64 or 128 (else FA_ERR_UNSUPPORTED).
  *   causal    0 or 1.
  *   scale     > 0 and finite; pass 0 (or any value <= 0) for 1/sqrt(d).  NaN/inf -> INVALID_ARG.
@@ -90,8 +90,8 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, fa_out_dt
  *   q            bf16 [B, H, Nq, d];  k, v: bf16 [B, H, Nk, d];  16-byte aligned.
  *   o            [B, H, Nq, d], bf16 or fp32 per o_dtype (fp32 for partials to be merged);
  *                lse: fp32 [B, H, Nq] or NULL (needed for merging).  Must not overlap the inputs.
- *   B, H, Nq, Nk >= 1;  0 <= q_row0 < Nq;  k_pos0 >= 0;  d: 64 or 128;  causal 0/1;  scale as for
- *   fa_fwd.
+ *   B, H, Nq, Nk >= 1;  B*H*ceil(Nq/256) < 2^31;  0 <= q_row0 < Nq;  k_pos0 >= 0;  d: 64 or 128;
+ *   causal 0/1;  scale as for fa_fwd.
  * Returns FA_OK once the kernels are queued.
  */
 fa_status fa_fwd_keyrange(const void *q, const void *k, const void *v, void *o, fa_out_dtype o_dtype,

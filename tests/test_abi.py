@@ -60,6 +60,11 @@ def test_fwd_rejects_bad_arguments(lib):
     # output overlapping an input
     assert fwd(lib, o=A + 16) == 1
     assert fwd(lib, lse=2 * A + 64) == 1
+    # more work units (pairs of 128-row query tiles) than an int counts: B*H = 2^30, 64 pairs each
+    # (buffers far apart, so only the unit count is wrong)
+    far = 1 << 52
+    assert lib.fa_fwd(far, 2 * far, 3 * far, 4 * far, 0, None, 1 << 15, 1 << 15, 1 << 14, 64, 0,
+                      0.0, None) == 1
 
 
 def dec(lib, ws=8 * A, ws_bytes=1 << 30, S=2, H=2, d=128, maxb=4, P=8, table=5 * A, lens=6 * A,
@@ -140,6 +145,9 @@ def test_keyrange_and_merge_rejections(lib):
                                    causal, 0.0, None)
     assert kr(q_row0=100) == 1 and kr(q_row0=-1) == 1 and kr(Nk=0) == 1 and kr(k_pos0=-5) == 1
     assert kr(causal=2) == 1 and kr(d=32) == 2
+    far = 1 << 52  # unit count past an int, buffers far apart
+    assert lib.fa_fwd_keyrange(far, 2 * far, 3 * far, 4 * far, 1, None, 1 << 15, 1 << 15, 1 << 14, 0,
+                               64, 0, 128, 0, 0.0, None) == 1
     assert kr(o=A + 64) == 1  # output overlaps q
     assert lib.fa_fwd_keyrange(A, 2 * A, 3 * A, 7 * A, 1, 2 * A + 64, 1, 2, 100, 0, 64, 0, 128, 0,
                                0.0, None) == 1  # LSE overlaps k
